@@ -1,0 +1,218 @@
+/*
+ * spear.h -- C ABI of the B200 (sm_100a) W4A16 linear layer with a
+ * per-token-gated low-rank Error Compensator (EC).
+ *
+ * The operation (SPEAR, gist.science technical summary, section 2.1 A
+ * "Compensateurs d'erreurs adaptatifs a l'entree": an EC projects the input
+ * into a low-rank space with A, gates it per token and projects back with B,
+ * on top of the 4-bit weight; fugumt.com abstract of arXiv 2606.11244: ECs
+ * "modulated by per-token gates" over W4 per-channel weights), in the
+ * row-vector scalar-gate form implemented here:
+ *
+ *     g_m = sigmoid(x_m . w_g + b_g)
+ *     y_m = x_m . dequant(W4) + g_m * ((x_m . A) . B)
+ *
+ *   x    M x K   bf16, row-major (token-major)
+ *   W    K x N   logically; stored as N output channels x K int4 codes
+ *   A    K x r   bf16,  B  r x N  bf16,  w_g  K  bf16,  b_g  float
+ *   y    M x N   bf16, row-major
+ *
+ * Conventions for every call below:
+ *   - bf16 and fp16 tensors are passed as uint16_t bit patterns.
+ *   - "device" pointers must point to CUDA device memory of the current
+ *     device; "host" pointers to ordinary host memory.  Device pointers must be
+ *     16-byte aligned (SPEAR_ERR_ALIGNMENT otherwise).
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls that launch work are asynchronous on that stream and return after
+ *     enqueueing.
+ *   - The caller owns every buffer.  No call allocates device memory.
+ *   - Arguments are validated before anything is enqueued; on error nothing
+ *     is launched and the call returns a nonzero SPEAR_* status, with a
+ *     message available from spear_last_error() (per host thread).  No call
+ *     aborts or exits the process.
+ *   - Shapes: K and N multiples of 128; r in {0, 16, 32, 64, 128}; group 0
+ *     (one fp16 scale per output channel) or 128 (one fp16 scale per 128
+ *     consecutive k and output channel); 1 <= M <= 65536.
+ */
+#ifndef SPEAR_H_
+#define SPEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------- */
+enum {
+  SPEAR_OK = 0,
+  SPEAR_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum   */
+  SPEAR_ERR_UNSUPPORTED_SHAPE = 2, /* K/N/r/group/M outside the list above    */
+  SPEAR_ERR_ALIGNMENT = 3,         /* a device pointer is not 16-byte aligned */
+  SPEAR_ERR_WORKSPACE = 4,         /* workspace smaller than required          */
+  SPEAR_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed     */
+  SPEAR_ERR_TIMEOUT = 6,           /* a device-side bounded wait expired       */
+  SPEAR_ERR_DEVICE_CHECK = 7       /* a device-side argument check failed      */
+};
+
+/* Kernel paths (for spear_linear_forward_path and the dispatcher). */
+enum {
+  SPEAR_PATH_AUTO = 0,    /* dispatcher's choice                                   */
+  SPEAR_PATH_DECODE = 1,  /* split-K GEMV kernel with the EC fused (M <= 16)       */
+  SPEAR_PATH_FUSED = 2,   /* tcgen05 GEMM with the EC fused into the same kernel   */
+  SPEAR_PATH_UNFUSED = 3  /* GEMM with the EC disabled, then a separate EC kernel  */
+};
+
+/* Message of the last failing call on this host thread ("" if none). */
+const char* spear_last_error(void);
+/* Static name of a status code. */
+const char* spear_status_string(int status);
+/* Library version, major*10000 + minor*100 + patch. */
+int spear_version(void);
+
+/* ---- sizes ---------------------------------------------------------------- */
+/* Bytes of a packed N x K int4 weight: N*K/2 (0 on a bad shape). */
+size_t spear_w4_packed_bytes(int N, int K);
+/* Number of fp16 scales: N (group 0) or (K/128)*N (group 128); 0 on a bad shape. */
+size_t spear_scale_count(int N, int K, int group);
+
+/* ---- a-0: quantiser --------------------------------------------------------
+ * Symmetric round-to-nearest int4 (SPEAR evaluates RTN per-channel W4
+ * weights, gist.science technical summary, section 3.1).  For every output
+ * channel n (and, for group 128, every block of 128 consecutive k):
+ *     s = fp16_rne(max|w| / 7)   (fp32 arithmetic; saturated to 65504;
+ *                                 s == 0 becomes 1.0 with all codes 0)
+ *     q = clamp(rint_even(w / s), -7, 7)   (IEEE fp32 quotient)
+ * W       device fp32, K x N row-major (W[k*N + n]).
+ * q       device int8, N x K row-major (q[n*K + k]), written.
+ * scales  device fp16 bits, [N] or [K/128][N], written.
+ * Bit-exact and deterministic. */
+int spear_w4_quantize(const float* W, int K, int N, int group, int8_t* q,
+                      uint16_t* scales, void* stream);
+
+/* ---- a-1: packed int4 weight layout -----------------------------------------
+ * Packed int4 weight layout (the pages give none; this one is built so that
+ * one 128-bit load per lane yields whole tensor-core operand fragments and a
+ * 16-row x 64-k tile is one contiguous, 16-byte aligned 512-byte block):
+ *   tile (p, t), p = n / 16, t = k / 64, occupies bytes
+ *       [(p * (K/64) + t) * 512, +512);
+ *   inside a tile, lane L = 0..31 owns bytes [16L, 16L+16) as four
+ *   little-endian uint32 words w_s (s = 0..3) at byte 16L + 4s;
+ *   with rho = L / 4 and c = L % 4, nibble slot i = 0..7 of w_s (bits
+ *   4i..4i+3) holds the code of
+ *       n = 16p + rho + 8*(i & 1)
+ *       k = 64t + 16c + 4s + 2*((i & 3) >> 1) + (i >> 2)
+ *   stored offset-binary: u = q + 8 (0..15).
+ * Requires N % 16 == 0 and K % 64 == 0 (the layer calls need multiples of 128).
+ * q       device int8 N x K (codes in [-8, 7]; other values are masked to 4 bits)
+ * packed  device uint8 [N*K/2], written.  Bit-exact. */
+int spear_w4_pack(const int8_t* q, int N, int K, uint8_t* packed, void* stream);
+/* Inverse of spear_w4_pack: packed -> q (N x K int8 in [-8, 7]).  Bit-exact. */
+int spear_w4_unpack(const uint8_t* packed, int N, int K, int8_t* q, void* stream);
+
+/* ---- EC operands -------------------------------------------------------------
+ * Per-channel fold: B'[j][n] = bf16_rne(fp32(B[j][n] / s[n])), so that a
+ * kernel accumulates x.q and (g t).B' in one fp32 accumulator and applies s_n
+ * once.  B, Bp: device bf16 r x N row-major; scales: device fp16 [N].
+ * Bit-exact. */
+int spear_ec_prescale_B(const uint16_t* B, const uint16_t* scales, int r, int N,
+                        uint16_t* Bp, void* stream);
+
+/* Elements of the two EC operand arrays: AgT (r+1) x K and BpT N x r. */
+size_t spear_ec_agt_count(int K, int r);
+size_t spear_ec_bpt_count(int N, int r);
+
+/* EC operands in the kernels' layout (one-off per layer):
+ *   AgT = [A^T ; w_g]          (r+1) x K bf16 row-major: the r projection rows
+ *                               and the gate weight as one extra row;
+ *   BpT = (B')^T (group 0) or B^T (group 128), N x r bf16 row-major.
+ * A: device bf16 K x r; B: device bf16 r x N; w_g: device bf16 [K];
+ * scales: the layer's fp16 scales (read only for group 0).  Bit-exact. */
+int spear_ec_pack(const uint16_t* A, const uint16_t* B, const uint16_t* w_g,
+                  const uint16_t* scales, int K, int N, int r, int group,
+                  uint16_t* AgT, uint16_t* BpT, void* stream);
+
+/* ---- the layer ----------------------------------------------------------------- */
+typedef struct spear_layer {
+  int K;                   /* input features  (multiple of 128)                  */
+  int N;                   /* output features (multiple of 128)                  */
+  int group;               /* 0 = per-channel scales, 128 = group-wise scales    */
+  int r;                   /* EC rank; 0 disables the EC                         */
+  const uint8_t* w_packed; /* device, spear_w4_pack layout, N*K/2 bytes           */
+  const uint16_t* scales;  /* device fp16, spear_scale_count(N, K, group) values  */
+  const uint16_t* AgT;     /* device bf16 (r+1) x K from spear_ec_pack (r > 0)    */
+  const uint16_t* BpT;     /* device bf16 N x r from spear_ec_pack (r > 0)        */
+  float b_g;               /* gate bias                                           */
+  float gate_tau;          /* threshold of the gate-mask count; <= 0 means 0.1    */
+} spear_layer;
+
+/* Workspace bytes needed by spear_linear_forward* for any 1 <= M <= M_max
+ * (0 on invalid arguments).  The workspace holds split-K partials, the EC
+ * projection, arrival counters and a device status word. */
+size_t spear_workspace_bytes(const spear_layer* layer, int M_max);
+
+/* Put a freshly allocated workspace into its initial state (zeroes it on
+ * stream).  Needed once after allocation and after any SPEAR_ERR_TIMEOUT;
+ * the kernels leave it in that state after every successful call. */
+int spear_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* y = layer(x) (see the top of this file).
+ * x          device bf16 M x K;  y  device bf16 M x N, written.
+ * ws         device workspace of ws_bytes >= spear_workspace_bytes(layer, M),
+ *            initialised once by spear_workspace_init.  A workspace must not
+ *            be used by two calls that may run concurrently.
+ * gate_out   optional (NULL): device fp32 [M], receives g_m (0 when r == 0).
+ * mask_count optional (NULL): device int32, receives #{m : g_m < gate_tau}.
+ * The kernel path is chosen by the dispatcher (see spear_dispatch_choice).
+ * Device-side failures (a bounded wait that expired) are reported through
+ * the workspace's status word, read by spear_read_status. */
+int spear_linear_forward(const spear_layer* layer, const uint16_t* x, int M,
+                         uint16_t* y, void* ws, size_t ws_bytes, float* gate_out,
+                         int* mask_count, void* stream);
+
+/* As spear_linear_forward with an explicit SPEAR_PATH_* (tests, tuning). */
+int spear_linear_forward_path(const spear_layer* layer, const uint16_t* x, int M,
+                              uint16_t* y, void* ws, size_t ws_bytes,
+                              float* gate_out, int* mask_count, int path,
+                              void* stream);
+
+/* Synchronise stream, read and clear the workspace's device status word.
+ * *device_status receives SPEAR_OK or the first device-side error code. */
+int spear_read_status(void* ws, int* device_status, void* stream);
+
+/* ---- a-7: dispatcher ----------------------------------------------------------
+ * Phase-aware choice between the fused and the unfused EC path (SPEAR,
+ * gist.science technical summary, section 2.2 A "Dispatch de fusion de noyau
+ * adaptatif sensible a la phase": decode fuses the EC into the low-bit GEMM,
+ * prefill runs it as a separate kernel; the choice here comes from measured
+ * kernel times, the pages' latency tables of section 2.2 C).
+ * The table is keyed by (K, N, r, group, M bucket); M buckets are powers of
+ * two (M rounded up).  Before tuning: DECODE for M <= 16, else FUSED. */
+int spear_dispatch_choice(const spear_layer* layer, int M);
+
+/* Time every applicable path for each M in Ms[0..nM) with CUDA events
+ * (median of `reps` runs, each preceded by writing flush_bytes of the
+ * optional device buffer `flush` to evict L2) and record the fastest in the
+ * table.  x: device bf16 M_max x K input, y: device bf16 M_max x N scratch
+ * output (M_max = max of Ms).  times_us (optional host array [nM*3]) receives
+ * the median of each path (DECODE, FUSED, UNFUSED; negative = not run).
+ * Synchronises the stream. */
+int spear_dispatch_tune(const spear_layer* layer, const int* Ms, int nM,
+                        const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes,
+                        void* flush, size_t flush_bytes, int reps, float* times_us,
+                        void* stream);
+
+/* Set one table entry by hand (path is a SPEAR_PATH_* other than AUTO). */
+int spear_dispatch_set(int K, int N, int r, int group, int M, int path);
+/* Forget every table entry. */
+void spear_dispatch_clear(void);
+/* Save / load the table as text (host file path). */
+int spear_dispatch_save(const char* path);
+int spear_dispatch_load(const char* path);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPEAR_H_ */

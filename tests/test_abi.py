@@ -1,0 +1,127 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+that include/spear.h declares, and its host-side logic (size queries,
+argument validation, dispatch table) behaves as documented."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "spear.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_0-9]+\**\s+\**(spear_[A-Za-z_0-9]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def S():
+    from w4_gemm_gated_b200 import build
+    build.build()
+    from w4_gemm_gated_b200 import spear
+    return spear
+
+
+def test_header_declares_expected_api():
+    names = _header_functions()
+    for must in ["spear_w4_quantize", "spear_w4_pack", "spear_w4_unpack", "spear_ec_prescale_B", "spear_ec_pack",
+                 "spear_workspace_bytes", "spear_linear_forward", "spear_linear_forward_path",
+                 "spear_dispatch_tune", "spear_dispatch_choice", "spear_dispatch_save", "spear_dispatch_load"]:
+        assert must in names
+
+
+def test_library_exports_every_header_symbol(S):
+    lib = ctypes.CDLL(S.LIB_PATH)
+    for name in _header_functions():
+        assert hasattr(lib, name), name
+    # and the binding declares a prototype for each of them
+    assert set(_header_functions()) <= set(S.EXPORTS)
+
+
+def test_size_queries(S):
+    assert S.F["spear_w4_packed_bytes"](11008, 4096) == 11008 * 4096 // 2
+    assert S.F["spear_w4_packed_bytes"](10, 64) == 0
+    assert S.F["spear_scale_count"](512, 512, 0) == 512
+    assert S.F["spear_scale_count"](4096, 14336, 128) == 112 * 4096
+    assert S.F["spear_scale_count"](4096, 100, 128) == 0
+    assert S.F["spear_ec_agt_count"](4096, 64) == 65 * 4096
+    assert S.F["spear_ec_bpt_count"](11008, 64) == 11008 * 64
+    assert S.version() >= 100
+    assert S.F["spear_status_string"](S.ERR_WORKSPACE) == b"SPEAR_ERR_WORKSPACE"
+
+
+def _layer(S, **kw):
+    d = dict(K=512, N=512, group=0, r=16, w_packed=0x10000, scales=0x20000, AgT=0x30000, BpT=0x40000,
+             b_g=0.0, gate_tau=0.1)
+    d.update(kw)
+    return S.LayerStruct(d["K"], d["N"], d["group"], d["r"], d["w_packed"], d["scales"], d["AgT"], d["BpT"],
+                         d["b_g"], d["gate_tau"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(K=500), 2), (dict(N=130), 2), (dict(r=8), 2), (dict(group=64), 2),
+    (dict(w_packed=None), 1), (dict(AgT=None), 1), (dict(scales=0x20008), 3),
+])
+def test_forward_validation_before_launch(S, kw, code):
+    st = _layer(S, **kw)
+    rc = S.F["spear_linear_forward"](ctypes.byref(st), 0x50000, 4, 0x60000, 0x70000, 1 << 30, None, None, None)
+    assert rc == code
+    assert S.F["spear_last_error"]().decode()
+
+
+def test_forward_rejects_bad_m_and_pointers(S):
+    st = _layer(S)
+    F = S.F["spear_linear_forward_path"]
+    assert F(ctypes.byref(st), 0x50000, 0, 0x60000, 0x70000, 1 << 30, None, None, 0, None) == S.ERR_UNSUPPORTED_SHAPE
+    assert F(ctypes.byref(st), None, 4, 0x60000, 0x70000, 1 << 30, None, None, 0, None) == S.ERR_INVALID_ARG
+    assert F(ctypes.byref(st), 0x50004, 4, 0x60000, 0x70000, 1 << 30, None, None, 0, None) == S.ERR_ALIGNMENT
+    assert F(ctypes.byref(st), 0x50000, 4, 0x60000, 0x70000, 1 << 30, None, None, 9, None) == S.ERR_INVALID_ARG
+    assert F(ctypes.byref(st), 0x50000, 32, 0x60000, 0x70000, 1 << 30, None, None, S.PATH_DECODE, None) \
+        == S.ERR_UNSUPPORTED_SHAPE
+    assert F(ctypes.byref(st), 0x50000, 4, 0x60000, 0x70000, 16, None, None, 0, None) == S.ERR_WORKSPACE
+
+
+def test_prep_calls_validate(S):
+    assert S.F["spear_w4_pack"](None, 16, 64, 0x1000, None) == S.ERR_INVALID_ARG
+    assert S.F["spear_w4_pack"](0x1000, 15, 64, 0x2000, None) == S.ERR_UNSUPPORTED_SHAPE
+    assert S.F["spear_w4_unpack"](0x1000, 16, 60, 0x2000, None) == S.ERR_UNSUPPORTED_SHAPE
+    assert S.F["spear_w4_quantize"](0x1000, 512, 512, 64, 0x2000, 0x3000, None) == S.ERR_UNSUPPORTED_SHAPE
+    assert S.F["spear_ec_pack"](0x1000, 0x2000, 0x3000, 0x4000, 512, 512, 24, 0, 0x5000, 0x6000, None) \
+        == S.ERR_UNSUPPORTED_SHAPE
+
+
+def test_workspace_bytes_grows_with_m(S):
+    st = _layer(S, K=4096, N=11008, r=64)
+    a = S.F["spear_workspace_bytes"](ctypes.byref(st), 16)
+    b = S.F["spear_workspace_bytes"](ctypes.byref(st), 2048)
+    assert 0 < a < b
+    assert S.F["spear_workspace_bytes"](ctypes.byref(st), 0) == 0
+
+
+def test_dispatch_table_default_set_save_load(S, tmp_path):
+    S.dispatch_clear()
+    st = _layer(S, K=4096, N=4096, r=64)
+    choice = S.F["spear_dispatch_choice"]
+    assert choice(ctypes.byref(st), 1) == S.PATH_DECODE
+    assert choice(ctypes.byref(st), 16) == S.PATH_DECODE
+    assert choice(ctypes.byref(st), 17) == S.PATH_FUSED
+    S.dispatch_set(4096, 4096, 64, 0, 100, S.PATH_UNFUSED)     # bucket 128
+    assert choice(ctypes.byref(st), 65) == S.PATH_UNFUSED
+    assert choice(ctypes.byref(st), 128) == S.PATH_UNFUSED
+    assert choice(ctypes.byref(st), 129) == S.PATH_FUSED
+    with pytest.raises(S.SpearError):
+        S.dispatch_set(4096, 4096, 64, 0, 64, S.PATH_DECODE)   # decode only up to M = 16
+    p = str(tmp_path / "lut.txt")
+    S.dispatch_save(p)
+    S.dispatch_clear()
+    assert choice(ctypes.byref(st), 100) == S.PATH_FUSED
+    S.dispatch_load(p)
+    assert choice(ctypes.byref(st), 100) == S.PATH_UNFUSED
+    bad = tmp_path / "bad.txt"
+    bad.write_text("1 2 3\n")
+    with pytest.raises(S.SpearError):
+        S.dispatch_load(str(bad))
+    S.dispatch_clear()

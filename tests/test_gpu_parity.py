@@ -1,0 +1,268 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
+
+Integer and byte work (quantiser codes and scales, packed bytes, EC operand
+layouts, gate-mask counts) must match bit for bit; floating-point outputs
+must satisfy max|y - y_ref| <= 1e-2 * max|y_ref| (bf16 output, fp32
+accumulation), the layer's stated error bound.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import spear_oracle as O
+from w4_gemm_gated_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+GATE_TOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def S():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from w4_gemm_gated_b200 import build
+    build.build()
+    from w4_gemm_gated_b200 import spear
+    return spear
+
+
+def dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def host_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def prepared(S, L: synth.LayerInputs, group: int, b_g=None):
+    W = torch.from_numpy(L.W).cuda()
+    A = dev_bf16(L.A) if L.r else None
+    B = dev_bf16(L.B) if L.r else None
+    wg = dev_bf16(L.w_g) if L.r else None
+    layer = S.prepare_layer(W, group, A, B, wg, L.b_g if b_g is None else b_g)
+    return layer
+
+
+def oracle_ref(L: synth.LayerInputs, group: int, b_g=None, x=None):
+    q, s = O.quantize_rtn(L.W, group)
+    y, g = O.linear(L.x if x is None else x, q, s, group, L.A, L.B, L.w_g, L.b_g if b_g is None else b_g)
+    return y, g, q, s
+
+
+def assert_close(y_gpu: torch.Tensor, y_ref: np.ndarray, tol=TOL):
+    yg = O.bf16_to_f64(host_bits(y_gpu))
+    assert yg.shape == y_ref.shape
+    assert np.all(np.isfinite(yg))
+    err = np.max(np.abs(yg - y_ref))
+    bound = tol * np.max(np.abs(y_ref))
+    assert err <= bound, f"max err {err:.3e} > {bound:.3e}"
+    return err / np.max(np.abs(y_ref))
+
+
+def run(S, layer, x_bits, path, M_max=None, gate=False):
+    x = dev_bf16(x_bits)
+    M = x.shape[0]
+    ws = S.make_workspace(layer, M_max or M)
+    g = torch.zeros(M, dtype=torch.float32, device="cuda") if gate else None
+    cnt = torch.zeros(1, dtype=torch.int32, device="cuda") if gate else None
+    y = S.forward(layer, x, ws, gate_out=g, mask_count=cnt, path=path)
+    torch.cuda.synchronize()
+    assert S.read_status(ws) == S.OK
+    return y, g, cnt, ws
+
+
+# ----------------------------------------------------------------------------
+# one-off preparation: bit-exact
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("group", [0, 128])
+@pytest.mark.parametrize("shape", [(512, 512), (4096, 11008)])
+def test_quantize_and_pack_bitexact(S, group, shape):
+    K, N = shape
+    L = synth.make_layer(1, K, N, 0, seed=3)
+    W = torch.from_numpy(L.W).cuda()
+    q, s = S.quantize(W, group)
+    qo, so = O.quantize_rtn(L.W, group)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), so.view(np.uint16))
+    p = S.pack(q)
+    assert np.array_equal(p.cpu().numpy(), O.pack_w4(qo))
+    assert torch.equal(S.unpack(p, N, K), q)
+
+
+def test_quantize_edge_channels(S):
+    # zero channel, saturating channel, subnormal-scale channel, exact ties
+    K, N = 128, 32
+    W = np.zeros((K, N), dtype=np.float32)
+    W[0, 1], W[1, 1] = 1e6, 5e5
+    W[0, 2] = 7e-7
+    W[:6, 3] = [7.0, 2.5, 3.5, -2.5, -0.5, 0.5]
+    W[:, 4] = np.linspace(-3, 3, K, dtype=np.float32)
+    q, s = S.quantize(torch.from_numpy(W).cuda(), 0)
+    qo, so = O.quantize_rtn(W, 0)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), so.view(np.uint16))
+
+
+def test_pack_all_codes_roundtrip(S):
+    rng = np.random.default_rng(5)
+    q = rng.integers(-8, 8, size=(256, 1024)).astype(np.int8)
+    p = S.pack(torch.from_numpy(q).cuda())
+    assert np.array_equal(p.cpu().numpy(), O.pack_w4(q))
+    assert np.array_equal(S.unpack(p, 256, 1024).cpu().numpy(), q)
+
+
+@pytest.mark.parametrize("group", [0, 128])
+def test_ec_pack_and_fold_bitexact(S, group):
+    L = synth.make_layer(1, 1024, 768, 64, seed=7)
+    qo, so = O.quantize_rtn(L.W, group)
+    s_dev = torch.from_numpy(so).cuda()
+    AgT, BpT = S.ec_pack(dev_bf16(L.A), dev_bf16(L.B), dev_bf16(L.w_g), s_dev, group)
+    AgT_o, BpT_o = O.ec_pack(L.A, L.B, L.w_g, so, group)
+    assert np.array_equal(host_bits(AgT), AgT_o)
+    assert np.array_equal(host_bits(BpT), BpT_o)
+    if group == 0:
+        Bp = S.prescale_B(dev_bf16(L.B), s_dev)
+        assert np.array_equal(host_bits(Bp), O.prescale_B(L.B, so))
+
+
+# ----------------------------------------------------------------------------
+# decode path (M <= 16)
+# ----------------------------------------------------------------------------
+
+def test_decode_tiny_config(S):
+    L = synth.tiny()
+    layer = prepared(S, L, 0)
+    y, g, cnt, _ = run(S, layer, L.x, S.PATH_DECODE, gate=True)
+    y_ref, g_ref, _, _ = oracle_ref(L, 0)
+    assert_close(y, y_ref)
+    assert np.max(np.abs(g.cpu().numpy() - g_ref)) <= GATE_TOL
+
+
+@pytest.fixture(scope="module")
+def decode_layer(S):
+    L = synth.decode(16, force_outlier=True)
+    return L, prepared(S, L, 0)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_decode_config_parity(S, decode_layer, M):
+    L, layer = decode_layer
+    Lm = synth.decode(M, force_outlier=True)
+    assert np.array_equal(Lm.W, L.W)
+    y, g, cnt, _ = run(S, layer, Lm.x, S.PATH_DECODE, gate=True)
+    y_ref, g_ref, _, _ = oracle_ref(Lm, 0)
+    assert_close(y, y_ref)
+    assert np.max(np.abs(g.cpu().numpy() - g_ref)) <= GATE_TOL
+    # gate-mask count: exact, tokens whose logit sits at the threshold excepted
+    _, logit = O.gate(Lm.x, Lm.w_g, Lm.b_g)
+    xf = O.bf16_to_f64(Lm.x)
+    band = 1e-3 * (1 + np.abs(xf) @ np.abs(O.bf16_to_f64(Lm.w_g)))
+    amb = np.abs(logit - math.log(0.1 / 0.9)) < band
+    lo = O.gate_mask_count(g_ref[~amb])
+    assert lo <= int(cnt.item()) <= lo + int(amb.sum())
+
+
+@pytest.mark.parametrize("M", [2, 3, 7, 9, 13])
+def test_decode_ragged_tokens(S, M):
+    L = synth.make_layer(M, 1024, 1536, 32, b_g=-0.5, x_kind="outlier", seed=11, force_outlier=True)
+    layer = prepared(S, L, 0)
+    y, _, _, _ = run(S, layer, L.x, S.PATH_DECODE)
+    assert_close(y, oracle_ref(L, 0)[0])
+
+
+@pytest.mark.parametrize("r", [16, 32, 64, 128])
+def test_decode_every_rank(S, r):
+    L = synth.make_layer(8, 2048, 2048, r, b_g=0.3, seed=20 + r)
+    layer = prepared(S, L, 0)
+    y, _, _, _ = run(S, layer, L.x, S.PATH_DECODE)
+    assert_close(y, oracle_ref(L, 0)[0])
+
+
+@pytest.mark.parametrize("shape", [(4096, 4096), (4096, 14336), (14336, 4096), (11008, 4096)])
+def test_decode_model_shapes(S, shape):
+    K, N = shape
+    L = synth.make_layer(16, K, N, 64, b_g=-1.0, x_kind="t3", seed=31)
+    layer = prepared(S, L, 0)
+    y, _, _, _ = run(S, layer, L.x, S.PATH_DECODE)
+    assert_close(y, oracle_ref(L, 0)[0])
+
+
+def test_decode_group128(S):
+    L = synth.make_layer(16, 4096, 4096, 64, b_g=-1.0, x_kind="outlier", seed=41, force_outlier=True)
+    layer = prepared(S, L, 128)
+    y, _, _, _ = run(S, layer, L.x, S.PATH_DECODE)
+    assert_close(y, oracle_ref(L, 128)[0])
+
+
+def test_decode_ec_disabled_invariants(S):
+    L = synth.make_layer(16, 2048, 2048, 64, b_g=0.5, seed=51)
+    W = torch.from_numpy(L.W).cuda()
+    plain = S.prepare_layer(W, 0, None, None, None, 0.0)
+    y0, _, _, _ = run(S, plain, L.x, S.PATH_DECODE)
+    y0_ref, _ = O.linear(L.x, *O.quantize_rtn(L.W, 0), 0, None, None, None, 0.0)
+    assert_close(y0, y0_ref)
+    # b_g = -inf: gate 0 -> exactly the EC-disabled output (values; +0 == -0)
+    off = prepared(S, L, 0, b_g=-math.inf)
+    y1, g1, _, _ = run(S, off, L.x, S.PATH_DECODE, gate=True)
+    assert torch.equal(y1.float(), y0.float())
+    assert torch.all(g1 == 0)
+    # A = 0 and B = 0 give the same
+    for zero in ("A", "B"):
+        Lz = synth.make_layer(16, 2048, 2048, 64, b_g=0.5, seed=51)
+        setattr(Lz, zero, np.zeros_like(getattr(Lz, zero)))
+        yz, _, _, _ = run(S, prepared(S, Lz, 0), L.x, S.PATH_DECODE)
+        assert torch.equal(yz.float(), y0.float())
+
+
+def test_decode_is_deterministic(S, decode_layer):
+    L, layer = decode_layer
+    x = dev_bf16(L.x)
+    ws = S.make_workspace(layer, 16)
+    ys = [S.forward(layer, x, ws, path=S.PATH_DECODE).clone() for _ in range(3)]
+    torch.cuda.synchronize()
+    assert all(torch.equal(ys[0].view(torch.int16), t.view(torch.int16)) for t in ys[1:])
+
+
+def test_oracle_packed_bytes_drive_the_gpu(S):
+    # the oracle's own reading of the packed layout, fed to the kernel
+    L = synth.make_layer(8, 1024, 1024, 32, b_g=0.1, seed=61)
+    q, s = O.quantize_rtn(L.W, 0)
+    AgT, BpT = O.ec_pack(L.A, L.B, L.w_g, s, 0)
+    layer = S.layer_from_parts(1024, 1024, 0, torch.from_numpy(O.pack_w4(q)).cuda(), torch.from_numpy(s).cuda(),
+                               dev_bf16(AgT), dev_bf16(BpT), L.b_g)
+    y, _, _, _ = run(S, layer, L.x, S.PATH_DECODE)
+    assert_close(y, O.linear(L.x, q, s, 0, L.A, L.B, L.w_g, L.b_g)[0])
+
+
+# ----------------------------------------------------------------------------
+# unfused path (EC-disabled GEMM, then the standalone EC kernel)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("group", [0, 128])
+def test_unfused_small_m(S, group):
+    L = synth.make_layer(16, 4096, 2048, 64, b_g=-1.0, x_kind="outlier", seed=71, force_outlier=True)
+    layer = prepared(S, L, group)
+    y, g, cnt, _ = run(S, layer, L.x, S.PATH_UNFUSED, gate=True)
+    y_ref, g_ref, _, _ = oracle_ref(L, group)
+    assert_close(y, y_ref)
+    assert np.max(np.abs(g.cpu().numpy() - g_ref)) <= GATE_TOL
+
+
+def test_workspace_reuse_across_paths_and_sizes(S):
+    # one workspace, several calls of different M and paths in a row
+    L = synth.make_layer(16, 2048, 2048, 64, b_g=-0.2, seed=81)
+    layer = prepared(S, L, 0)
+    ws = S.make_workspace(layer, 16)
+    q, s = O.quantize_rtn(L.W, 0)
+    for M, path in [(16, S.PATH_DECODE), (3, S.PATH_UNFUSED), (9, S.PATH_DECODE), (16, S.PATH_UNFUSED),
+                    (1, S.PATH_DECODE)]:
+        x = L.x[:M]
+        y = S.forward(layer, dev_bf16(x), ws, path=path)
+        torch.cuda.synchronize()
+        assert_close(y, O.linear(x, q, s, 0, L.A, L.B, L.w_g, L.b_g)[0])
+    assert S.read_status(ws) == S.OK

@@ -1,0 +1,523 @@
+// C ABI of the library (declared in include/spear.h): argument validation,
+// workspace layout, the measured-time dispatch table and path selection.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace spear {
+
+static thread_local std::string g_last_error;
+
+int set_error(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int set_cuda_error(const char* what, cudaError_t e) {
+  return set_error(SPEAR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int sm_count() {
+  static std::mutex mu;
+  static std::map<int, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    dev = -1;  // no usable device: size plans for a full B200
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(dev);
+  if (it != cache.end()) return it->second;
+  int n = 0;
+  if (dev < 0 || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = 148;
+  }
+  cache[dev] = n;
+  return n;
+}
+
+static bool valid_r(int r) { return r == 0 || r == 16 || r == 32 || r == 64 || r == 128; }
+
+static int check_kn(int K, int N) {
+  if (K <= 0 || N <= 0 || K % 128 || N % 128)
+    return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "K=%d N=%d: both must be positive multiples of 128", K, N);
+  if ((long long)K * N > (1LL << 34)) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "K*N too large");
+  return SPEAR_OK;
+}
+
+static int check_layer(const spear_layer* l, LayerView* out) {
+  if (!l) return set_error(SPEAR_ERR_INVALID_ARG, "layer is NULL");
+  int rc = check_kn(l->K, l->N);
+  if (rc) return rc;
+  if (l->group != 0 && l->group != 128)
+    return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "group=%d: must be 0 or 128", l->group);
+  if (!valid_r(l->r)) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "r=%d: must be 0, 16, 32, 64 or 128", l->r);
+  if (!l->w_packed || !l->scales) return set_error(SPEAR_ERR_INVALID_ARG, "w_packed / scales is NULL");
+  if (l->r > 0 && (!l->AgT || !l->BpT)) return set_error(SPEAR_ERR_INVALID_ARG, "r > 0 needs AgT and BpT");
+  if (!aligned16(l->w_packed) || !aligned16(l->scales) || (l->r > 0 && (!aligned16(l->AgT) || !aligned16(l->BpT))))
+    return set_error(SPEAR_ERR_ALIGNMENT, "layer device pointers must be 16-byte aligned");
+  out->K = l->K;
+  out->N = l->N;
+  out->group = l->group;
+  out->r = l->r;
+  out->w = l->w_packed;
+  out->scales = reinterpret_cast<const __half*>(l->scales);
+  out->agt = l->r > 0 ? reinterpret_cast<const __nv_bfloat16*>(l->AgT) : nullptr;
+  out->bpt = l->r > 0 ? reinterpret_cast<const __nv_bfloat16*>(l->BpT) : nullptr;
+  out->b_g = l->b_g;
+  out->tau = l->gate_tau > 0.f ? l->gate_tau : 0.1f;
+  return SPEAR_OK;
+}
+
+// ---------------------------------------------------------------------------
+// workspace layout
+// ---------------------------------------------------------------------------
+struct WsLayout {
+  size_t hdr, mflags, tickets, tcflags, t, gt, part, total;
+  int n_flags;
+};
+
+static size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+static WsLayout ws_layout_uncached(const LayerView& L, int M_max) {
+  WsLayout w = {};
+  const int Mpad = ((M_max + 127) / 128) * 128;
+  const int RT = 32 * ((L.r / 16 + 2) / 2) + 16;  // >= decode (32*E2) and EC-kernel row strides
+  w.n_flags = Mpad / 16 + 64;
+  size_t off = kWsHeaderBytes;
+  w.hdr = 0;
+  w.mflags = off;
+  off = up256(off + sizeof(int) * w.n_flags);
+  w.tickets = off;
+  off = up256(off + sizeof(int) * w.n_flags);
+  w.tcflags = off;
+  off = up256(off + sizeof(int) * w.n_flags);
+  w.t = off;
+  off = up256(off + sizeof(float) * 16 * (size_t)RT);
+  w.gt = off;
+  off = up256(off + 2 * (size_t)Mpad * (L.r > 0 ? L.r : 1));
+  w.part = off;
+  size_t part_floats = 0;
+  if (L.r > 0) {
+    // largest partial buffer over every M <= M_max (the K split shrinks as M grows)
+    for (int M = 16; M <= M_max + 15; M += 16) {
+      EcPlan p = plan_ec(std::min(M, M_max), L.K, L.N, L.r, sm_count());
+      part_floats = std::max(part_floats, p.part_floats);
+    }
+  }
+  off = up256(off + sizeof(float) * part_floats);
+  w.total = off;
+  return w;
+}
+
+static WsLayout ws_layout(const LayerView& L, int M_max) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int, int, int>, WsLayout> cache;
+  const auto key = std::make_tuple(L.K, L.N, L.r, L.group, M_max, sm_count());
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  const WsLayout w = ws_layout_uncached(L, M_max);
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache.size() > 4096) cache.clear();
+  cache[key] = w;
+  return w;
+}
+
+// ---------------------------------------------------------------------------
+// dispatch table
+// ---------------------------------------------------------------------------
+using DKey = std::tuple<int, int, int, int, int>;  // K, N, r, group, M bucket
+static std::mutex g_dmu;
+static std::map<DKey, int> g_table;
+
+static int m_bucket(int M) {
+  int b = 1;
+  while (b < M) b <<= 1;
+  return b;
+}
+
+static int default_path(const LayerView& L, int M) {
+  (void)L;
+  return M <= 16 ? SPEAR_PATH_DECODE : SPEAR_PATH_FUSED;
+}
+
+static int choose_path(const LayerView& L, int M) {
+  {
+    std::lock_guard<std::mutex> lk(g_dmu);
+    auto it = g_table.find(DKey(L.K, L.N, L.r, L.group, m_bucket(M)));
+    if (it != g_table.end()) {
+      const int p = it->second;
+      if (!(p == SPEAR_PATH_DECODE && M > 16)) return p;
+    }
+  }
+  return default_path(L, M);
+}
+
+// ---------------------------------------------------------------------------
+// forward
+// ---------------------------------------------------------------------------
+static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, uint8_t* ws,
+                    const WsLayout& wl, float* gate_out, int* mask_count, int path, cudaStream_t st) {
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + wl.hdr);
+  int* mflags = reinterpret_cast<int*>(ws + wl.mflags);
+  int* tickets = reinterpret_cast<int*>(ws + wl.tickets);
+  int* tcflags = reinterpret_cast<int*>(ws + wl.tcflags);
+  float* tbuf = reinterpret_cast<float*>(ws + wl.t);
+  __nv_bfloat16* gt = reinterpret_cast<__nv_bfloat16*>(ws + wl.gt);
+  float* part = reinterpret_cast<float*>(ws + wl.part);
+  const int sms = sm_count();
+  if (path == SPEAR_PATH_DECODE) {
+    if (M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs M <= 16 (M=%d)", M);
+    DecodePlan p = plan_decode(M, L.K, L.N, L.r, L.group, sms);
+    const char* why = check_decode_plan(p);
+    if (why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", why);
+    return launch_decode(p, L, x, M, y, hdr, tbuf, gt, gate_out, mask_count, false, st);
+  }
+  if (path == SPEAR_PATH_UNFUSED) {
+    LayerView L0 = L;
+    L0.r = 0;
+    L0.agt = nullptr;
+    L0.bpt = nullptr;
+    int rc;
+    if (M <= 16) {
+      DecodePlan p = plan_decode(M, L.K, L.N, 0, L.group, sms);
+      const char* why = check_decode_plan(p);
+      if (why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", why);
+      rc = launch_decode(p, L0, x, M, y, hdr, tbuf, gt, L.r > 0 ? nullptr : gate_out,
+                         L.r > 0 ? nullptr : mask_count, false, st);
+      if (rc || L.r == 0) return rc;
+      // the separate EC launch: same kernel in EC-only mode, y += g (t . B) in place
+      DecodePlan pe = plan_decode(M, L.K, L.N, L.r, L.group, sms);
+      why = check_decode_plan(pe);
+      if (why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", why);
+      return launch_decode(pe, L, x, M, y, hdr, tbuf, gt, gate_out, mask_count, true, st);
+    } else {
+      TcPlan p = plan_tc(M, L.K, L.N, 0, L.group, sms);
+      rc = launch_tc(p, L0, x, M, y, false, hdr, tcflags, gt, L.r > 0 ? nullptr : gate_out,
+                     L.r > 0 ? nullptr : mask_count, st);
+    }
+    if (rc || L.r == 0) return rc;
+    EcPlan ep = plan_ec(M, L.K, L.N, L.r, sms);
+    return launch_ec(ep, L, x, M, y, hdr, part, tickets, mflags, gt, gate_out, mask_count, st);
+  }
+  if (path == SPEAR_PATH_FUSED) {
+    TcPlan p = plan_tc(M, L.K, L.N, L.r, L.group, sms);
+    return launch_tc(p, L, x, M, y, L.r > 0, hdr, tcflags, gt, gate_out, mask_count, st);
+  }
+  return set_error(SPEAR_ERR_INVALID_ARG, "unknown path %d", path);
+}
+
+static int forward_impl(const spear_layer* layer, const uint16_t* x, int M, uint16_t* y, void* ws, size_t ws_bytes,
+                        float* gate_out, int* mask_count, int path, void* stream) {
+  LayerView L;
+  int rc = check_layer(layer, &L);
+  if (rc) return rc;
+  if (M < 1 || M > 65536) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "M=%d outside [1, 65536]", M);
+  if (!x || !y || !ws) return set_error(SPEAR_ERR_INVALID_ARG, "x, y and ws must be non-NULL");
+  if (!aligned16(x) || !aligned16(y) || !aligned16(ws) || (gate_out && ((uintptr_t)gate_out & 3)) ||
+      (mask_count && ((uintptr_t)mask_count & 3)))
+    return set_error(SPEAR_ERR_ALIGNMENT, "x, y, ws must be 16-byte aligned");
+  if (path < SPEAR_PATH_AUTO || path > SPEAR_PATH_UNFUSED) return set_error(SPEAR_ERR_INVALID_ARG, "bad path %d", path);
+  const WsLayout wl = ws_layout(L, M);
+  if (ws_bytes < wl.total)
+    return set_error(SPEAR_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed for M=%d", ws_bytes, wl.total, M);
+  if (path == SPEAR_PATH_AUTO) path = choose_path(L, M);
+  if (path == SPEAR_PATH_DECODE && M > 16)
+    return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs M <= 16 (M=%d)", M);
+  return run_path(L, reinterpret_cast<const __nv_bfloat16*>(x), M, reinterpret_cast<__nv_bfloat16*>(y),
+                  static_cast<uint8_t*>(ws), wl, gate_out, mask_count, path, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace spear
+
+using namespace spear;
+
+extern "C" {
+
+const char* spear_last_error(void) { return g_last_error.c_str(); }
+
+const char* spear_status_string(int status) {
+  switch (status) {
+    case SPEAR_OK: return "SPEAR_OK";
+    case SPEAR_ERR_INVALID_ARG: return "SPEAR_ERR_INVALID_ARG";
+    case SPEAR_ERR_UNSUPPORTED_SHAPE: return "SPEAR_ERR_UNSUPPORTED_SHAPE";
+    case SPEAR_ERR_ALIGNMENT: return "SPEAR_ERR_ALIGNMENT";
+    case SPEAR_ERR_WORKSPACE: return "SPEAR_ERR_WORKSPACE";
+    case SPEAR_ERR_CUDA: return "SPEAR_ERR_CUDA";
+    case SPEAR_ERR_TIMEOUT: return "SPEAR_ERR_TIMEOUT";
+    case SPEAR_ERR_DEVICE_CHECK: return "SPEAR_ERR_DEVICE_CHECK";
+    default: return "SPEAR_ERR_UNKNOWN";
+  }
+}
+
+int spear_version(void) { return 100; }
+
+size_t spear_w4_packed_bytes(int N, int K) {
+  if (N <= 0 || K <= 0 || N % 16 || K % 64) return 0;
+  return (size_t)N * K / 2;
+}
+
+size_t spear_scale_count(int N, int K, int group) {
+  if (N <= 0 || K <= 0) return 0;
+  if (group == 0) return (size_t)N;
+  if (group == 128 && K % 128 == 0) return (size_t)(K / 128) * N;
+  return 0;
+}
+
+int spear_w4_quantize(const float* W, int K, int N, int group, int8_t* q, uint16_t* scales, void* stream) {
+  g_last_error.clear();
+  if (!W || !q || !scales) return set_error(SPEAR_ERR_INVALID_ARG, "NULL pointer");
+  if (K <= 0 || N <= 0 || K % 32 || N % 32)
+    return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "quantize needs K, N positive multiples of 32");
+  if (group != 0 && !(group == 128 && K % 128 == 0))
+    return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "group=%d with K=%d", group, K);
+  if (!aligned16(W) || !aligned16(q) || !aligned16(scales)) return set_error(SPEAR_ERR_ALIGNMENT, "unaligned pointer");
+  return launch_quantize(W, K, N, group, q, reinterpret_cast<__half*>(scales), static_cast<cudaStream_t>(stream));
+}
+
+int spear_w4_pack(const int8_t* q, int N, int K, uint8_t* packed, void* stream) {
+  g_last_error.clear();
+  if (!q || !packed) return set_error(SPEAR_ERR_INVALID_ARG, "NULL pointer");
+  if (N <= 0 || K <= 0 || N % 16 || K % 64)
+    return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "pack needs N %% 16 == 0 and K %% 64 == 0");
+  if (!aligned16(q) || !aligned16(packed)) return set_error(SPEAR_ERR_ALIGNMENT, "unaligned pointer");
+  return launch_pack(q, N, K, packed, static_cast<cudaStream_t>(stream));
+}
+
+int spear_w4_unpack(const uint8_t* packed, int N, int K, int8_t* q, void* stream) {
+  g_last_error.clear();
+  if (!q || !packed) return set_error(SPEAR_ERR_INVALID_ARG, "NULL pointer");
+  if (N <= 0 || K <= 0 || N % 16 || K % 64)
+    return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "unpack needs N %% 16 == 0 and K %% 64 == 0");
+  if (!aligned16(q) || !aligned16(packed)) return set_error(SPEAR_ERR_ALIGNMENT, "unaligned pointer");
+  return launch_unpack(packed, N, K, q, static_cast<cudaStream_t>(stream));
+}
+
+int spear_ec_prescale_B(const uint16_t* B, const uint16_t* scales, int r, int N, uint16_t* Bp, void* stream) {
+  g_last_error.clear();
+  if (!B || !scales || !Bp) return set_error(SPEAR_ERR_INVALID_ARG, "NULL pointer");
+  if (r <= 0 || N <= 0) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "r and N must be positive");
+  if (!aligned16(B) || !aligned16(scales) || !aligned16(Bp)) return set_error(SPEAR_ERR_ALIGNMENT, "unaligned pointer");
+  return launch_prescale(reinterpret_cast<const __nv_bfloat16*>(B), reinterpret_cast<const __half*>(scales), r, N,
+                         reinterpret_cast<__nv_bfloat16*>(Bp), false, static_cast<cudaStream_t>(stream));
+}
+
+size_t spear_ec_agt_count(int K, int r) { return (K > 0 && r > 0) ? (size_t)(r + 1) * K : 0; }
+size_t spear_ec_bpt_count(int N, int r) { return (N > 0 && r > 0) ? (size_t)N * r : 0; }
+
+int spear_ec_pack(const uint16_t* A, const uint16_t* B, const uint16_t* w_g, const uint16_t* scales, int K, int N,
+                  int r, int group, uint16_t* AgT, uint16_t* BpT, void* stream) {
+  g_last_error.clear();
+  if (!A || !B || !w_g || !AgT || !BpT || (group == 0 && !scales)) return set_error(SPEAR_ERR_INVALID_ARG, "NULL pointer");
+  int rc = check_kn(K, N);
+  if (rc) return rc;
+  if (r <= 0 || !valid_r(r)) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "r=%d", r);
+  if (group != 0 && group != 128) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "group=%d", group);
+  if (!aligned16(A) || !aligned16(B) || !aligned16(w_g) || !aligned16(AgT) || !aligned16(BpT))
+    return set_error(SPEAR_ERR_ALIGNMENT, "unaligned pointer");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = launch_agt(reinterpret_cast<const __nv_bfloat16*>(A), reinterpret_cast<const __nv_bfloat16*>(w_g), K, r,
+                  reinterpret_cast<__nv_bfloat16*>(AgT), st);
+  if (rc) return rc;
+  if (group == 0)
+    return launch_prescale(reinterpret_cast<const __nv_bfloat16*>(B), reinterpret_cast<const __half*>(scales), r, N,
+                           reinterpret_cast<__nv_bfloat16*>(BpT), true, st);
+  return launch_transpose_b(reinterpret_cast<const __nv_bfloat16*>(B), r, N, reinterpret_cast<__nv_bfloat16*>(BpT), st);
+}
+
+size_t spear_workspace_bytes(const spear_layer* layer, int M_max) {
+  LayerView L;
+  if (check_layer(layer, &L) != SPEAR_OK || M_max < 1 || M_max > 65536) return 0;
+  return ws_layout(L, M_max).total;
+}
+
+int spear_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (!ws || ws_bytes < kWsHeaderBytes) return set_error(SPEAR_ERR_INVALID_ARG, "bad workspace");
+  cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SPEAR_OK : set_cuda_error("workspace memset", e);
+}
+
+int spear_linear_forward(const spear_layer* layer, const uint16_t* x, int M, uint16_t* y, void* ws, size_t ws_bytes,
+                         float* gate_out, int* mask_count, void* stream) {
+  g_last_error.clear();
+  return forward_impl(layer, x, M, y, ws, ws_bytes, gate_out, mask_count, SPEAR_PATH_AUTO, stream);
+}
+
+int spear_linear_forward_path(const spear_layer* layer, const uint16_t* x, int M, uint16_t* y, void* ws,
+                              size_t ws_bytes, float* gate_out, int* mask_count, int path, void* stream) {
+  g_last_error.clear();
+  return forward_impl(layer, x, M, y, ws, ws_bytes, gate_out, mask_count, path, stream);
+}
+
+int spear_read_status(void* ws, int* device_status, void* stream) {
+  g_last_error.clear();
+  if (!ws || !device_status) return set_error(SPEAR_ERR_INVALID_ARG, "NULL pointer");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return set_cuda_error("stream synchronize", e);
+  int v = 0;
+  e = cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return set_cuda_error("status read", e);
+  if (v) {
+    const int zero = 0;
+    e = cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return set_cuda_error("status clear", e);
+  }
+  *device_status = v;
+  return SPEAR_OK;
+}
+
+int spear_dispatch_choice(const spear_layer* layer, int M) {
+  LayerView L;
+  if (check_layer(layer, &L) != SPEAR_OK || M < 1) return SPEAR_PATH_AUTO;
+  return choose_path(L, M);
+}
+
+int spear_dispatch_set(int K, int N, int r, int group, int M, int path) {
+  g_last_error.clear();
+  if (path < SPEAR_PATH_DECODE || path > SPEAR_PATH_UNFUSED) return set_error(SPEAR_ERR_INVALID_ARG, "bad path");
+  if (M < 1) return set_error(SPEAR_ERR_INVALID_ARG, "bad M");
+  if (path == SPEAR_PATH_DECODE && M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs M <= 16");
+  std::lock_guard<std::mutex> lk(g_dmu);
+  g_table[DKey(K, N, r, group, m_bucket(M))] = path;
+  return SPEAR_OK;
+}
+
+void spear_dispatch_clear(void) {
+  std::lock_guard<std::mutex> lk(g_dmu);
+  g_table.clear();
+}
+
+int spear_dispatch_save(const char* path) {
+  g_last_error.clear();
+  if (!path) return set_error(SPEAR_ERR_INVALID_ARG, "NULL path");
+  FILE* f = fopen(path, "w");
+  if (!f) return set_error(SPEAR_ERR_INVALID_ARG, "cannot open %s for writing", path);
+  std::lock_guard<std::mutex> lk(g_dmu);
+  fprintf(f, "# spear dispatch table v1: K N r group M_bucket path\n");
+  for (const auto& kv : g_table)
+    fprintf(f, "%d %d %d %d %d %d\n", std::get<0>(kv.first), std::get<1>(kv.first), std::get<2>(kv.first),
+            std::get<3>(kv.first), std::get<4>(kv.first), kv.second);
+  fclose(f);
+  return SPEAR_OK;
+}
+
+int spear_dispatch_load(const char* path) {
+  g_last_error.clear();
+  if (!path) return set_error(SPEAR_ERR_INVALID_ARG, "NULL path");
+  FILE* f = fopen(path, "r");
+  if (!f) return set_error(SPEAR_ERR_INVALID_ARG, "cannot open %s", path);
+  std::map<DKey, int> t;
+  char line[256];
+  int lineno = 0;
+  while (fgets(line, sizeof(line), f)) {
+    ++lineno;
+    if (line[0] == '#' || line[0] == '\n') continue;
+    int K, N, r, g, mb, p;
+    if (sscanf(line, "%d %d %d %d %d %d", &K, &N, &r, &g, &mb, &p) != 6 || p < SPEAR_PATH_DECODE ||
+        p > SPEAR_PATH_UNFUSED || mb < 1) {
+      fclose(f);
+      return set_error(SPEAR_ERR_INVALID_ARG, "%s:%d: malformed entry", path, lineno);
+    }
+    t[DKey(K, N, r, g, mb)] = p;
+  }
+  fclose(f);
+  std::lock_guard<std::mutex> lk(g_dmu);
+  for (const auto& kv : t) g_table[kv.first] = kv.second;
+  return SPEAR_OK;
+}
+
+int spear_dispatch_tune(const spear_layer* layer, const int* Ms, int nM, const uint16_t* x, uint16_t* y, void* ws,
+                        size_t ws_bytes, void* flush, size_t flush_bytes, int reps, float* times_us, void* stream) {
+  g_last_error.clear();
+  LayerView L;
+  int rc = check_layer(layer, &L);
+  if (rc) return rc;
+  if (!Ms || nM <= 0 || !x || !y || !ws) return set_error(SPEAR_ERR_INVALID_ARG, "NULL argument");
+  if (reps < 1) reps = 1;
+  int M_max = 0;
+  for (int i = 0; i < nM; ++i) {
+    if (Ms[i] < 1 || Ms[i] > 65536) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "bad M %d", Ms[i]);
+    M_max = std::max(M_max, Ms[i]);
+  }
+  const WsLayout wl = ws_layout(L, M_max);
+  if (ws_bytes < wl.total) return set_error(SPEAR_ERR_WORKSPACE, "workspace too small for M_max=%d", M_max);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaEvent_t e0, e1;
+  if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess)
+    return set_error(SPEAR_ERR_CUDA, "event create failed");
+  int result = SPEAR_OK;
+  for (int i = 0; i < nM && result == SPEAR_OK; ++i) {
+    const int M = Ms[i];
+    float best = 1e30f;
+    int best_path = default_path(L, M);
+    const int paths[3] = {SPEAR_PATH_DECODE, SPEAR_PATH_FUSED, SPEAR_PATH_UNFUSED};
+    for (int pi = 0; pi < 3; ++pi) {
+      const int path = paths[pi];
+      float med = -1.f;
+      if (!(path == SPEAR_PATH_DECODE && M > 16)) {
+        std::vector<float> ts;
+        int prc = SPEAR_OK;
+        for (int rep = 0; rep < reps + 2 && prc == SPEAR_OK; ++rep) {
+          if (flush && flush_bytes) cudaMemsetAsync(flush, rep & 0xff, flush_bytes, st);
+          cudaEventRecord(e0, st);
+          prc = run_path(L, reinterpret_cast<const __nv_bfloat16*>(x), M, reinterpret_cast<__nv_bfloat16*>(y),
+                         static_cast<uint8_t*>(ws), wl, nullptr, nullptr, path, st);
+          cudaEventRecord(e1, st);
+          if (prc == SPEAR_OK) {
+            cudaError_t ce = cudaEventSynchronize(e1);
+            if (ce != cudaSuccess) {
+              result = set_cuda_error("tune", ce);
+              break;
+            }
+            float ms = 0.f;
+            cudaEventElapsedTime(&ms, e0, e1);
+            if (rep >= 2) ts.push_back(ms * 1000.f);
+          }
+        }
+        if (result) break;
+        if (prc == SPEAR_OK && !ts.empty()) {
+          std::sort(ts.begin(), ts.end());
+          med = ts[ts.size() / 2];
+          if (med < best) {
+            best = med;
+            best_path = path;
+          }
+        } else {
+          g_last_error.clear();
+        }
+      }
+      if (times_us) times_us[i * 3 + pi] = med;
+    }
+    if (result == SPEAR_OK) {
+      std::lock_guard<std::mutex> lk(g_dmu);
+      g_table[DKey(L.K, L.N, L.r, L.group, m_bucket(M))] = best_path;
+    }
+  }
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  return result;
+}
+
+}  // extern "C"

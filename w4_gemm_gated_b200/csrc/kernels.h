@@ -1,0 +1,78 @@
+// Internal interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace spear {
+
+struct WsHeader;
+
+// Record a CUDA failure as the thread's last error; returns SPEAR_ERR_CUDA.
+int set_cuda_error(const char* what, cudaError_t e);
+// Record a message as the thread's last error; returns `code`.
+int set_error(int code, const char* fmt, ...);
+
+// A validated layer, with typed device pointers.
+struct LayerView {
+  int K, N, group, r;
+  const uint8_t* w;
+  const __half* scales;
+  const __nv_bfloat16* agt;  // (r+1) x K, or null when r == 0
+  const __nv_bfloat16* bpt;  // N x r, or null when r == 0
+  float b_g, tau;
+};
+
+// ---- decode path (decode.cu) ----
+struct DecodePlan {
+  int MT;       // token tile: 8 or 16
+  int CS;       // cluster size = number of K parts
+  int NC;       // clusters
+  int kt_part;  // 64-wide k-tiles per K part
+  int E2, P2;   // EC pairs, weight pairs
+  int RT;       // row stride of the EC projection buffer (32 * E2)
+  size_t smem;
+};
+DecodePlan plan_decode(int M, int K, int N, int r, int group, int sm_count);
+// 0 if the plan respects the kernel's static limits, else a message.
+const char* check_decode_plan(const DecodePlan& p);
+int launch_decode(const DecodePlan& p, const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y,
+                  WsHeader* hdr, float* ws_t, __nv_bfloat16* ws_gt, float* gate_out, int* mask_count, bool ec_only,
+                  cudaStream_t st);
+
+// ---- standalone EC kernel (ec.cu): y += g * (x.A).B, in place ----
+struct EcPlan {
+  int ksplit;   // K parts of the projection
+  int grid;     // persistent CTAs
+  int RT;       // row stride of projection partials
+  size_t part_floats;  // floats of the partial buffer
+};
+EcPlan plan_ec(int M, int K, int N, int r, int sm_count);
+int launch_ec(const EcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y,
+              WsHeader* hdr, float* part, int* tickets, int* mflags, __nv_bfloat16* gt, float* gate_out,
+              int* mask_count, cudaStream_t st);
+
+// ---- tensor-core path (tc_gemm.cu) ----
+struct TcPlan {
+  int grid;
+  int m_blocks, n_blocks;
+  size_t smem;
+};
+TcPlan plan_tc(int M, int K, int N, int r, int group, int sm_count);
+int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, bool with_ec,
+              WsHeader* hdr, int* mflags, __nv_bfloat16* gt, float* gate_out, int* mask_count, cudaStream_t st);
+
+// ---- packing kernels (pack.cu) ----
+int launch_quantize(const float* W, int K, int N, int group, int8_t* q, __half* s, cudaStream_t st);
+int launch_pack(const int8_t* q, int N, int K, uint8_t* packed, cudaStream_t st);
+int launch_unpack(const uint8_t* packed, int N, int K, int8_t* q, cudaStream_t st);
+int launch_prescale(const __nv_bfloat16* B, const __half* s, int r, int N, __nv_bfloat16* Bp, bool transpose,
+                    cudaStream_t st);
+int launch_agt(const __nv_bfloat16* A, const __nv_bfloat16* w_g, int K, int r, __nv_bfloat16* AgT,
+               cudaStream_t st);
+int launch_transpose_b(const __nv_bfloat16* B, int r, int N, __nv_bfloat16* BT, cudaStream_t st);
+
+}  // namespace spear

@@ -1,0 +1,600 @@
+// Tensor-core path (M > 16): persistent tcgen05 W4A16 GEMM with the gated EC
+// fused into the same kernel.
+//
+// SPEAR fuses the EC work into the low-bit GEMM (gist.science technical
+// summary, section 2.2 A and B: the post-EC computation folded into the
+// GEMM epilogue).  On sm_100a this kernel does, per 128-token x 256-channel
+// output tile:
+//   * a TMA producer warp streams the x tile (128 x 64 bf16, 128-byte
+//     swizzle) and the packed int4 tile (256 channels x 64 k, 8 KB: sixteen
+//     512-byte tiles of the packed layout, one 3-D tensor-map box);
+//   * eight dequant warps turn the int4 tile into bf16 in shared memory, in
+//     the UMMA canonical K-major 128-byte-swizzled layout (exact small
+//     integers for per-channel scales; s * q rounded once for group scales);
+//   * one MMA warp issues tcgen05.mma (kind::f16, M=128, N=256, K=16) into a
+//     double-buffered fp32 accumulator in tensor memory;
+//   * four epilogue warps read the accumulator with tcgen05.ld, apply the
+//     per-channel scale and store bf16 y.
+// The EC: the first tiles of the schedule are "projection tiles"
+// [t | logit] = x . [A | w_g] (N = r+16 columns through the same pipeline);
+// their epilogue applies the gate, writes gt = g * t (bf16) and raises an
+// epoch-tagged flag per 128-token block.  Every output tile then runs
+// ceil(r/64) extra K-steps, gt (128 x r) times (B')^T (256 x r), into the
+// same accumulator (B' = B / s_n is folded once per layer, so s_n applies
+// to the sum), so the EC costs neither a second kernel nor a pass over y.
+//
+// Every wait on an mbarrier or a flag is bounded; on expiry the kernel
+// records SPEAR_ERR_TIMEOUT and all roles leave their loops.
+#include <cuda.h>
+
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace spear {
+
+constexpr int TC_BM = 128;
+constexpr int TC_BN = 256;
+constexpr int TC_BK = 64;
+constexpr int TC_STAGES = 3;
+constexpr int TC_THREADS = 14 * 32;  // producer, mma, 4 epilogue, 8 dequant warps
+constexpr int TC_X_BYTES = TC_BM * TC_BK * 2;      // 16 KB
+constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;      // 32 KB
+constexpr int TC_P_BYTES = TC_BN * TC_BK / 2;      // 8 KB
+constexpr int TC_STAGE_BYTES = TC_X_BYTES + TC_B_BYTES + TC_P_BYTES;
+constexpr int TC_SMEM = TC_STAGES * TC_STAGE_BYTES + 1024 /* barriers */ + 1024 /* alignment */;
+
+struct TcArgs {
+  const __half* scales;
+  __nv_bfloat16* y;
+  float* gate_out;
+  int* mask_count;
+  WsHeader* hdr;
+  int* mflags;        // per 128-token block: +1 per epilogue warp once its gt rows are out
+  __nv_bfloat16* gt;  // [Mb * 128][r]
+  int M, K, N, r, group;
+  float b_g, tau;
+  int Mb, Nb;       // 128-token blocks, 256-channel blocks
+  int with_ec;      // projection tiles + EC k-steps
+  int NE;           // projection tile width: 16 * ceil((r + 1) / 16)
+  int ec_steps;     // ceil(r / 64)
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait; false after a timeout or once another role has given up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, WsHeader* h) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      report_status(h, SPEAR_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint64_t* bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          dst),
+      "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint64_t* bar, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
+          "r"(dst),
+      "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// SW128 K-major UMMA shared-memory descriptor (8-row groups 1024 bytes apart).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;            // leading byte offset (16 B; unused with 128-byte swizzle)
+  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset: next 8-row group
+  d |= (uint64_t)1 << 46;            // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;            // 128-byte swizzle
+  return d;
+}
+
+// kind::f16 instruction descriptor: bf16 x bf16 -> fp32, both K-major.
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+
+// ---------------------------------------------------------------------------
+// schedule shared by all roles
+// ---------------------------------------------------------------------------
+struct TileInfo {
+  int kind;  // 0 = projection tile, 1 = output tile
+  int mb, nb;
+  int steps;  // k-steps of this tile
+};
+
+__device__ __forceinline__ TileInfo tile_info(const TcArgs& a, int tile) {
+  TileInfo t;
+  const int KT = a.K / TC_BK;
+  const int nproj = a.with_ec ? a.Mb : 0;
+  if (tile < nproj) {
+    t.kind = 0;
+    t.mb = tile;
+    t.nb = 0;
+    t.steps = KT;
+  } else {
+    const int i = tile - nproj;
+    t.kind = 1;
+    t.mb = i / a.Nb;
+    t.nb = i % a.Nb;
+    t.steps = KT + (a.with_ec ? a.ec_steps : 0);
+  }
+  return t;
+}
+
+// int4 tile (16 strips of 512 B) -> bf16 [256 rows][64 k] in the SW128 K-major layout.
+template <bool GROUP>
+__device__ __forceinline__ void dequant_tile(const uint8_t* psrc, uint8_t* bdst, int dt, const TcArgs& a, int nb,
+                                             int kt) {
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int chunk = dt + it * 256;          // 512 chunks of 16 bytes
+    const int strip = chunk >> 5, L = chunk & 31;
+    const int rho = L >> 2, c = L & 3;
+    const uint4 w = *reinterpret_cast<const uint4*>(psrc + chunk * 16);
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+    uint32_t o[4][4];  // o[s][pi]
+#pragma unroll
+    for (int s = 0; s < 4; ++s) int4x8_to_bf16x8(wv[s], o[s]);
+    const int n0 = strip * 16 + rho;  // row within the 256-row tile
+    const int n1 = n0 + 8;
+    if (GROUP) {
+      // bf16(s * q), rounded once: q * s = q * s_hi + q * s_lo with s_hi = bf16(s)
+      const int g = kt / 2;
+      const float s0 = __half2float(a.scales[(size_t)g * a.N + nb * TC_BN + n0]);
+      const float s1 = __half2float(a.scales[(size_t)g * a.N + nb * TC_BN + n1]);
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(s0), h1 = __float2bfloat16_rn(s1);
+      const __nv_bfloat162 hi0 = __halves2bfloat162(h0, h0), hi1 = __halves2bfloat162(h1, h1);
+      const __nv_bfloat16 l0 = __float2bfloat16_rn(s0 - __bfloat162float(h0));
+      const __nv_bfloat16 l1 = __float2bfloat16_rn(s1 - __bfloat162float(h1));
+      const __nv_bfloat162 lo0 = __halves2bfloat162(l0, l0), lo1 = __halves2bfloat162(l1, l1);
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+#pragma unroll
+        for (int pi = 0; pi < 4; ++pi) {
+          const bool row1 = pi & 1;
+          __nv_bfloat162 q = *reinterpret_cast<__nv_bfloat162*>(&o[s][pi]);
+          const __nv_bfloat162 p = __hmul2(q, row1 ? lo1 : lo0);
+          q = __hfma2(q, row1 ? hi1 : hi0, p);
+          o[s][pi] = *reinterpret_cast<uint32_t*>(&q);
+        }
+      }
+    }
+    // row n0: k 16c + 4s + {0,1} = o[s][0], {2,3} = o[s][2];  row n1: o[s][1], o[s][3]
+    const int ch0 = 2 * c, ch1 = 2 * c + 1;  // 16-byte chunks of the 128-byte row
+    uint8_t* r0 = bdst + (n0 >> 3) * 1024 + (n0 & 7) * 128;
+    uint8_t* r1 = bdst + (n1 >> 3) * 1024 + (n1 & 7) * 128;
+    *reinterpret_cast<uint4*>(r0 + ((ch0 ^ (n0 & 7)) << 4)) = make_uint4(o[0][0], o[0][2], o[1][0], o[1][2]);
+    *reinterpret_cast<uint4*>(r0 + ((ch1 ^ (n0 & 7)) << 4)) = make_uint4(o[2][0], o[2][2], o[3][0], o[3][2]);
+    *reinterpret_cast<uint4*>(r1 + ((ch0 ^ (n1 & 7)) << 4)) = make_uint4(o[0][1], o[0][3], o[1][1], o[1][3]);
+    *reinterpret_cast<uint4*>(r1 + ((ch1 ^ (n1 & 7)) << 4)) = make_uint4(o[2][1], o[2][3], o[3][1], o[3][3]);
+  }
+}
+
+template <bool GROUP>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    tc_kernel(const __grid_constant__ TcArgs a, const __grid_constant__ CUtensorMap tm_x,
+              const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_agt,
+              const __grid_constant__ CUtensorMap tm_bpt, const __grid_constant__ CUtensorMap tm_gt) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* xs = smem;                                        // [STAGES][16 KB]
+  uint8_t* bs = smem + TC_STAGES * TC_X_BYTES;               // [STAGES][32 KB]
+  uint8_t* ps = bs + TC_STAGES * TC_B_BYTES;                 // [STAGES][8 KB]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + TC_STAGES * TC_P_BYTES);
+  uint64_t* full = bars;                     // TMA loads of a stage landed
+  uint64_t* ready = bars + TC_STAGES;        // B operand of a stage ready (dequant warps)
+  uint64_t* empty = bars + 2 * TC_STAGES;    // MMAs of a stage done
+  uint64_t* acc_full = bars + 3 * TC_STAGES; // [2]
+  uint64_t* acc_empty = acc_full + 2;        // [2]
+  uint32_t* tmem_base_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int epoch = *reinterpret_cast<volatile int*>(&a.hdr->epoch);
+  const int ntiles = (a.with_ec ? a.Mb : 0) + a.Mb * a.Nb;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < TC_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&ready[s], 8);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_base_holder)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_holder;
+  if (!a.with_ec && blockIdx.x == 0) {
+    // EC disabled: every gate is 0, below any positive threshold
+    if (a.gate_out)
+      for (int m = threadIdx.x; m < a.M; m += blockDim.x) a.gate_out[m] = 0.f;
+    if (a.mask_count && threadIdx.x == 0) *a.mask_count = a.M;
+  }
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const TileInfo ti = tile_info(a, tile);
+        const int KT = a.K / TC_BK;
+        for (int k = 0; k < ti.steps && ok; ++k) {
+          ok = mbar_wait(&empty[s], ph ^ 1, abort_flag, a.hdr);
+          if (!ok) break;
+          uint8_t* xd = xs + s * TC_X_BYTES;
+          uint8_t* bd = bs + s * TC_B_BYTES;
+          uint8_t* pd = ps + s * TC_P_BYTES;
+          if (ti.kind == 0) {
+            mbar_arrive_tx(&full[s], TC_X_BYTES + a.NE * 128);
+            tma_load_2d(smem_u32(xd), &tm_x, &full[s], k * TC_BK, ti.mb * TC_BM);
+            tma_load_2d(smem_u32(bd), &tm_agt, &full[s], k * TC_BK, 0);
+          } else if (k < KT) {
+            mbar_arrive_tx(&full[s], TC_X_BYTES + TC_P_BYTES);
+            tma_load_2d(smem_u32(xd), &tm_x, &full[s], k * TC_BK, ti.mb * TC_BM);
+            tma_load_3d(smem_u32(pd), &tm_w, &full[s], 0, k, ti.nb * (TC_BN / 16));
+          } else {
+            const int e = k - KT;
+            if (e == 0) {
+              // gated projection of this token block must be published
+              ok = wait_flag_eq(&a.mflags[ti.mb], 4 * (epoch + 1), a.hdr);
+              if (!ok) {
+                *abort_flag = 1;
+                break;
+              }
+              asm volatile("fence.proxy.async.global;" ::: "memory");
+            }
+            mbar_arrive_tx(&full[s], TC_X_BYTES + TC_B_BYTES);
+            tma_load_2d(smem_u32(xd), &tm_gt, &full[s], e * TC_BK, ti.mb * TC_BM);
+            tma_load_2d(smem_u32(bd), &tm_bpt, &full[s], e * TC_BK, ti.nb * TC_BN);
+          }
+          if (++s == TC_STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int buf = 0;
+      uint32_t aph[2] = {0, 0};
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const TileInfo ti = tile_info(a, tile);
+        ok = mbar_wait(&acc_empty[buf], aph[buf] ^ 1, abort_flag, a.hdr);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + buf * 256;
+        const uint32_t idesc = ti.kind == 0 ? make_idesc(TC_BM, a.NE) : make_idesc(TC_BM, TC_BN);
+        for (int k = 0; k < ti.steps && ok; ++k) {
+          ok = mbar_wait(&ready[s], ph, abort_flag, a.hdr);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t ad = sw128_desc(smem_u32(xs + s * TC_X_BYTES));
+          const uint64_t bd = sw128_desc(smem_u32(bs + s * TC_B_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < TC_BK / 16; ++kk)
+            umma(d, ad + 2 * kk, bd + 2 * kk, idesc, (k > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&empty[s]);
+          if (++s == TC_STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[buf]);
+        aph[buf] ^= 1;
+        buf ^= 1;
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter of this warp
+    int buf = 0;
+    uint32_t aph[2] = {0, 0};
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      const TileInfo ti = tile_info(a, tile);
+      ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], aph[buf], abort_flag, a.hdr));
+      if (!ok) break;
+      tc_fence_after();
+      const int row = q * 32 + lane;
+      const int m = ti.mb * TC_BM + row;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * 256;
+      if (ti.kind == 0) {
+        // projection tile: columns 0..r-1 = t, column r = gate logit
+        float lv[16];
+        tmem_ld16(taddr + (a.r / 16) * 16, lv);
+        const float g = sigmoidf_(lv[0] + a.b_g);
+        const bool valid = m < a.M;
+        if (valid && a.gate_out) a.gate_out[m] = g;
+        const unsigned below = __ballot_sync(0xffffffffu, valid && g < a.tau);
+        if (lane == 0 && a.mask_count && below) atomicAdd(&a.hdr->ec_done, __popc(below));
+        __nv_bfloat16* gdst = a.gt + (size_t)m * a.r;
+        for (int c0 = 0; c0 < a.r; c0 += 16) {
+          float tv[16];
+          tmem_ld16(taddr + c0, tv);
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(g * tv[2 * i], g * tv[2 * i + 1]);
+          uint4* d4 = reinterpret_cast<uint4*>(gdst + c0);
+          d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+        tc_fence_before();
+        __syncwarp();
+        // four epilogue warps per block: the block is ready at 4 * (epoch + 1)
+        if (lane == 0) atomicAdd(&a.mflags[ti.mb], 1);
+      } else {
+        const int n0 = ti.nb * TC_BN;
+#pragma unroll 1
+        for (int c0 = 0; c0 < TC_BN; c0 += 16) {
+          float v[16];
+          tmem_ld16(taddr + c0, v);
+          if (!GROUP) {
+            const uint4* sp = reinterpret_cast<const uint4*>(a.scales + n0 + c0);
+            const uint4 s0 = __ldg(sp), s1 = __ldg(sp + 1);
+            const __half* h0 = reinterpret_cast<const __half*>(&s0);
+            const __half* h1 = reinterpret_cast<const __half*>(&s1);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              v[i] *= __half2float(h0[i]);
+              v[8 + i] *= __half2float(h1[i]);
+            }
+          }
+          if (m < a.M) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+            uint4* dst = reinterpret_cast<uint4*>(a.y + (size_t)m * a.N + n0 + c0);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+        tc_fence_before();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      aph[buf] ^= 1;
+      buf ^= 1;
+    }
+  } else {
+    // ------------------------------------------------------------ dequant
+    const int dt = threadIdx.x - 6 * 32;  // 0..255
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      const TileInfo ti = tile_info(a, tile);
+      const int KT = a.K / TC_BK;
+      for (int k = 0; k < ti.steps && ok; ++k) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, a.hdr));
+        if (!ok) break;
+        if (ti.kind == 1 && k < KT) {
+          dequant_tile<GROUP>(ps + s * TC_P_BYTES, bs + s * TC_B_BYTES, dt, a, ti.nb, k);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ready[s]);
+        if (++s == TC_STAGES) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512));
+  }
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int prev = atomicAdd(&a.hdr->done_ctas, 1);
+    if (prev == (int)gridDim.x - 1) {
+      if (a.mask_count && a.with_ec) *a.mask_count = a.hdr->ec_done;
+      a.hdr->done_ctas = 0;
+      a.hdr->ec_done = 0;
+      __threadfence();
+      atomicAdd(&a.hdr->epoch, 1);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+static bool tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                         uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// packed weight as a 3-D array of 32-bit words: [N/16 strips][K/64 tiles][128 words]
+static bool tmap_packed(CUtensorMap* m, const void* base, int K, int N) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {128, (cuuint64_t)(K / 64), (cuuint64_t)(N / 16)};
+  const cuuint64_t strides[2] = {512, (cuuint64_t)(K / 64) * 512};
+  const cuuint32_t box[3] = {128, 1, TC_BN / 16};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+TcPlan plan_tc(int M, int K, int N, int r, int group, int sm_count) {
+  (void)K;
+  (void)r;
+  (void)group;
+  TcPlan p = {};
+  p.m_blocks = (M + TC_BM - 1) / TC_BM;
+  p.n_blocks = N / TC_BN;
+  p.grid = sm_count;
+  p.smem = TC_SMEM;
+  return p;
+}
+
+template <bool GROUP>
+static int launch_tc_t(const TcPlan& p, const TcArgs& a, const CUtensorMap* maps, cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(tc_kernel<GROUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+  });
+  if (attr_err != cudaSuccess) return set_cuda_error("cudaFuncSetAttribute(tc)", attr_err);
+  const int ntiles = (a.with_ec ? a.Mb : 0) + a.Mb * a.Nb;
+  const int grid = ntiles < p.grid ? ntiles : p.grid;
+  tc_kernel<GROUP><<<grid, TC_THREADS, p.smem, st>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4]);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SPEAR_OK : set_cuda_error("tc kernel launch", e);
+}
+
+int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, bool with_ec,
+              WsHeader* hdr, int* mflags, __nv_bfloat16* gt, float* gate_out, int* mask_count, cudaStream_t st) {
+  if (L.N % TC_BN) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "tensor-core path needs N %% 256 == 0 (N=%d)", L.N);
+  TcArgs a = {};
+  a.scales = L.scales;
+  a.y = y;
+  a.gate_out = gate_out;
+  a.mask_count = mask_count;
+  a.hdr = hdr;
+  a.mflags = mflags;
+  a.gt = gt;
+  a.M = M;
+  a.K = L.K;
+  a.N = L.N;
+  a.r = with_ec ? L.r : 0;
+  a.group = L.group;
+  a.b_g = L.b_g;
+  a.tau = L.tau;
+  a.Mb = p.m_blocks;
+  a.Nb = p.n_blocks;
+  a.with_ec = with_ec && L.r > 0;
+  a.NE = 16 * ((a.r + 1 + 15) / 16);
+  a.ec_steps = (a.r + TC_BK - 1) / TC_BK;
+  CUtensorMap maps[5];
+  memset(maps, 0, sizeof(maps));
+  bool ok = tmap_2d_bf16(&maps[0], x, L.K, M, TC_BK, TC_BM) && tmap_packed(&maps[1], L.w, L.K, L.N);
+  if (ok && a.with_ec) {
+    ok = tmap_2d_bf16(&maps[2], L.agt, L.K, L.r + 1, TC_BK, a.NE) &&
+         tmap_2d_bf16(&maps[3], L.bpt, L.r, L.N, TC_BK, TC_BN) &&
+         tmap_2d_bf16(&maps[4], gt, L.r, (uint64_t)p.m_blocks * TC_BM, TC_BK, TC_BM);
+  }
+  if (!ok) return set_error(SPEAR_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  return L.group ? launch_tc_t<true>(p, a, maps, st) : launch_tc_t<false>(p, a, maps, st);
+}
+
+}  // namespace spear

@@ -1,0 +1,285 @@
+"""ctypes binding of ``libspear.so`` (C ABI in ``include/spear.h``).
+
+Argument marshalling only: every step of the layer runs in the CUDA library.
+PyTorch tensors supply device memory and the current CUDA stream.  Importing
+this module loads the library and raises ``ImportError`` if it is missing;
+there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspear.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m w4_gemm_gated_b200.build`")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_UNSUPPORTED_SHAPE = 2
+ERR_ALIGNMENT = 3
+ERR_WORKSPACE = 4
+ERR_CUDA = 5
+ERR_TIMEOUT = 6
+ERR_DEVICE_CHECK = 7
+
+PATH_AUTO = 0
+PATH_DECODE = 1
+PATH_FUSED = 2
+PATH_UNFUSED = 3
+PATH_NAMES = {PATH_DECODE: "decode", PATH_FUSED: "fused", PATH_UNFUSED: "unfused"}
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+_f = ctypes.c_float
+
+
+class LayerStruct(ctypes.Structure):
+    """Mirror of ``spear_layer``."""
+
+    _fields_ = [
+        ("K", _i), ("N", _i), ("group", _i), ("r", _i),
+        ("w_packed", _vp), ("scales", _vp), ("AgT", _vp), ("BpT", _vp),
+        ("b_g", _f), ("gate_tau", _f),
+    ]
+
+
+def _proto(name, restype, *argtypes):
+    fn = getattr(_lib, name)
+    fn.restype = restype
+    fn.argtypes = list(argtypes)
+    return fn
+
+
+EXPORTS = {
+    "spear_last_error": (ctypes.c_char_p,),
+    "spear_status_string": (ctypes.c_char_p, _i),
+    "spear_version": (_i,),
+    "spear_w4_packed_bytes": (_sz, _i, _i),
+    "spear_scale_count": (_sz, _i, _i, _i),
+    "spear_w4_quantize": (_i, _vp, _i, _i, _i, _vp, _vp, _vp),
+    "spear_w4_pack": (_i, _vp, _i, _i, _vp, _vp),
+    "spear_w4_unpack": (_i, _vp, _i, _i, _vp, _vp),
+    "spear_ec_prescale_B": (_i, _vp, _vp, _i, _i, _vp, _vp),
+    "spear_ec_agt_count": (_sz, _i, _i),
+    "spear_ec_bpt_count": (_sz, _i, _i),
+    "spear_ec_pack": (_i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp),
+    "spear_workspace_bytes": (_sz, ctypes.POINTER(LayerStruct), _i),
+    "spear_workspace_init": (_i, _vp, _sz, _vp),
+    "spear_linear_forward": (_i, ctypes.POINTER(LayerStruct), _vp, _i, _vp, _vp, _sz, _vp, _vp, _vp),
+    "spear_linear_forward_path": (_i, ctypes.POINTER(LayerStruct), _vp, _i, _vp, _vp, _sz, _vp, _vp, _i, _vp),
+    "spear_read_status": (_i, _vp, ctypes.POINTER(_i), _vp),
+    "spear_dispatch_choice": (_i, ctypes.POINTER(LayerStruct), _i),
+    "spear_dispatch_tune": (_i, ctypes.POINTER(LayerStruct), ctypes.POINTER(_i), _i, _vp, _vp, _vp, _sz, _vp, _sz,
+                            _i, ctypes.POINTER(_f), _vp),
+    "spear_dispatch_set": (_i, _i, _i, _i, _i, _i, _i),
+    "spear_dispatch_clear": (None,),
+    "spear_dispatch_save": (_i, ctypes.c_char_p),
+    "spear_dispatch_load": (_i, ctypes.c_char_p),
+}
+
+F = {name: _proto(name, sig[0], *sig[1:]) for name, sig in EXPORTS.items()}
+LIB_PATH = _LIB_PATH
+
+
+class SpearError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{F['spear_status_string'](status).decode()}: {msg}")
+        self.status = status
+
+
+def _check(rc: int) -> None:
+    if rc != OK:
+        raise SpearError(rc, F["spear_last_error"]().decode())
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream: torch.cuda.Stream | None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def version() -> int:
+    return F["spear_version"]()
+
+
+# --------------------------------------------------------------------------
+# one-off layer preparation
+# --------------------------------------------------------------------------
+
+def quantize(W: torch.Tensor, group: int = 0, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """W (K x N fp32, device) -> codes q (N x K int8) and fp16 scales."""
+    K, N = W.shape
+    q = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    ns = F["spear_scale_count"](N, K, group)
+    if ns == 0:
+        raise SpearError(ERR_UNSUPPORTED_SHAPE, f"bad shape K={K} N={N} group={group}")
+    s = torch.empty(ns if group == 0 else (K // 128, N), dtype=torch.float16, device=W.device)
+    _check(F["spear_w4_quantize"](_ptr(W), K, N, group, _ptr(q), _ptr(s), _stream(stream)))
+    return q, s
+
+
+def pack(q: torch.Tensor, stream=None) -> torch.Tensor:
+    N, K = q.shape
+    out = torch.empty(N * K // 2, dtype=torch.uint8, device=q.device)
+    _check(F["spear_w4_pack"](_ptr(q), N, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def unpack(packed: torch.Tensor, N: int, K: int, stream=None) -> torch.Tensor:
+    q = torch.empty((N, K), dtype=torch.int8, device=packed.device)
+    _check(F["spear_w4_unpack"](_ptr(packed), N, K, _ptr(q), _stream(stream)))
+    return q
+
+
+def prescale_B(B: torch.Tensor, s: torch.Tensor, stream=None) -> torch.Tensor:
+    r, N = B.shape
+    out = torch.empty_like(B)
+    _check(F["spear_ec_prescale_B"](_ptr(B), _ptr(s), r, N, _ptr(out), _stream(stream)))
+    return out
+
+
+def ec_pack(A: torch.Tensor, B: torch.Tensor, w_g: torch.Tensor, s: torch.Tensor, group: int,
+            stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    K, r = A.shape
+    N = B.shape[1]
+    AgT = torch.empty((r + 1, K), dtype=torch.bfloat16, device=A.device)
+    BpT = torch.empty((N, r), dtype=torch.bfloat16, device=A.device)
+    _check(F["spear_ec_pack"](_ptr(A), _ptr(B), _ptr(w_g), _ptr(s), K, N, r, group, _ptr(AgT), _ptr(BpT),
+                              _stream(stream)))
+    return AgT, BpT
+
+
+@dataclass
+class Layer:
+    """Device-resident prepared layer (keeps its tensors alive)."""
+
+    K: int
+    N: int
+    group: int
+    r: int
+    w_packed: torch.Tensor
+    scales: torch.Tensor
+    AgT: torch.Tensor | None
+    BpT: torch.Tensor | None
+    b_g: float
+    gate_tau: float = 0.1
+
+    def struct(self) -> LayerStruct:
+        return LayerStruct(self.K, self.N, self.group, self.r, _ptr(self.w_packed), _ptr(self.scales),
+                           _ptr(self.AgT) if self.AgT is not None else None,
+                           _ptr(self.BpT) if self.BpT is not None else None,
+                           float(self.b_g), float(self.gate_tau))
+
+
+def prepare_layer(W: torch.Tensor, group: int, A: torch.Tensor | None, B: torch.Tensor | None,
+                  w_g: torch.Tensor | None, b_g: float, gate_tau: float = 0.1, stream=None) -> Layer:
+    """Quantise, pack and lay out one layer on the device (all steps in CUDA)."""
+    K, N = W.shape
+    q, s = quantize(W, group, stream)
+    w_packed = pack(q, stream)
+    del q
+    if A is not None:
+        AgT, BpT = ec_pack(A, B, w_g, s, group, stream)
+        r = A.shape[1]
+    else:
+        AgT = BpT = None
+        r = 0
+    return Layer(K, N, group, r, w_packed, s, AgT, BpT, b_g, gate_tau)
+
+
+def layer_from_parts(K: int, N: int, group: int, w_packed: torch.Tensor, scales: torch.Tensor,
+                     AgT: torch.Tensor | None, BpT: torch.Tensor | None, b_g: float,
+                     gate_tau: float = 0.1) -> Layer:
+    r = 0 if AgT is None else AgT.shape[0] - 1
+    return Layer(K, N, group, r, w_packed, scales, AgT, BpT, b_g, gate_tau)
+
+
+# --------------------------------------------------------------------------
+# forward
+# --------------------------------------------------------------------------
+
+def workspace_bytes(layer: Layer, M_max: int) -> int:
+    st = layer.struct()
+    n = F["spear_workspace_bytes"](ctypes.byref(st), M_max)
+    if n == 0:
+        raise SpearError(ERR_INVALID_ARG, "spear_workspace_bytes rejected the layer / M_max")
+    return n
+
+
+def make_workspace(layer: Layer, M_max: int, device=None, stream=None) -> torch.Tensor:
+    n = workspace_bytes(layer, M_max)
+    ws = torch.empty(n, dtype=torch.uint8, device=device or layer.w_packed.device)
+    _check(F["spear_workspace_init"](_ptr(ws), n, _stream(stream)))
+    return ws
+
+
+def forward(layer: Layer, x: torch.Tensor, ws: torch.Tensor, y: torch.Tensor | None = None,
+            gate_out: torch.Tensor | None = None, mask_count: torch.Tensor | None = None,
+            path: int = PATH_AUTO, stream=None) -> torch.Tensor:
+    """y = x . dequant(W4) + g * ((x . A) . B) for x (M x K bf16) on the device."""
+    M, K = x.shape
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bf16")
+    if y is None:
+        y = torch.empty((M, layer.N), dtype=torch.bfloat16, device=x.device)
+    st = layer.struct()
+    _check(F["spear_linear_forward_path"](ctypes.byref(st), _ptr(x), M, _ptr(y), _ptr(ws), ws.numel(),
+                                          _ptr(gate_out), _ptr(mask_count), path, _stream(stream)))
+    return y
+
+
+def read_status(ws: torch.Tensor, stream=None) -> int:
+    v = _i(0)
+    _check(F["spear_read_status"](_ptr(ws), ctypes.byref(v), _stream(stream)))
+    return v.value
+
+
+# --------------------------------------------------------------------------
+# dispatcher
+# --------------------------------------------------------------------------
+
+def dispatch_choice(layer: Layer, M: int) -> int:
+    st = layer.struct()
+    return F["spear_dispatch_choice"](ctypes.byref(st), M)
+
+
+def dispatch_tune(layer: Layer, Ms: list[int], x: torch.Tensor, y: torch.Tensor, ws: torch.Tensor,
+                  flush: torch.Tensor | None = None, reps: int = 20, stream=None) -> list[tuple[float, float, float]]:
+    st = layer.struct()
+    arr = (_i * len(Ms))(*Ms)
+    times = (_f * (3 * len(Ms)))()
+    _check(F["spear_dispatch_tune"](ctypes.byref(st), arr, len(Ms), _ptr(x), _ptr(y), _ptr(ws), ws.numel(),
+                                    _ptr(flush), 0 if flush is None else flush.numel() * flush.element_size(),
+                                    reps, times, _stream(stream)))
+    return [(times[3 * i], times[3 * i + 1], times[3 * i + 2]) for i in range(len(Ms))]
+
+
+def dispatch_set(K: int, N: int, r: int, group: int, M: int, path: int) -> None:
+    _check(F["spear_dispatch_set"](K, N, r, group, M, path))
+
+
+def dispatch_clear() -> None:
+    F["spear_dispatch_clear"]()
+
+
+def dispatch_save(path: str) -> None:
+    _check(F["spear_dispatch_save"](path.encode()))
+
+
+def dispatch_load(path: str) -> None:
+    _check(F["spear_dispatch_load"](path.encode()))
