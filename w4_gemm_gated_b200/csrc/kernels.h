@@ -34,6 +34,7 @@ struct DecodePlan {
   int kt_part;  // 64-wide k-tiles per K part
   int E2, P2;   // EC pairs, weight pairs
   int RT;       // row stride of the EC projection buffer (32 * E2)
+  int ring;     // 4 KB shared-memory ring slots
   size_t smem;
 };
 DecodePlan plan_decode(int M, int K, int N, int r, int group, int sm_count);
