@@ -121,3 +121,25 @@ def test_fused_is_deterministic(S):
     torch.cuda.synchronize()
     assert all(torch.equal(ys[0].view(torch.int16), t.view(torch.int16)) for t in ys[1:])
     assert S.read_status(ws) == S.OK
+
+
+def test_one_workspace_across_paths_and_sizes(S):
+    # the same workspace serves every path and size in any order (its flags are
+    # epoch-tagged per launch, so no call can see another call's state)
+    L = synth.make_layer(640, 2048, 1024, 64, b_g=-0.3, seed=600)
+    layer = prepared(S, L, 0)
+    ws = S.make_workspace(layer, 640)
+    q, s = O.quantize_rtn(L.W, 0)
+    plain = S.Layer(layer.K, layer.N, 0, 0, layer.w_packed, layer.scales, None, None, 0.0)
+    order = [(128, S.PATH_FUSED), (128, S.PATH_UNFUSED), (16, S.PATH_DECODE), (512, S.PATH_FUSED),
+             (640, S.PATH_UNFUSED), (300, S.PATH_FUSED), (5, S.PATH_UNFUSED), (640, S.PATH_FUSED),
+             (40, S.PATH_UNFUSED), (600, S.PATH_UNFUSED), (16, S.PATH_UNFUSED), (256, S.PATH_UNFUSED)]
+    for it, (M, path) in enumerate(order):
+        x = L.x[:M]
+        if it % 3 == 2:
+            # an EC-disabled layer on the same workspace in between
+            S.forward(plain, dev_bf16(x), ws, path=S.PATH_FUSED)
+        y = S.forward(layer, dev_bf16(x), ws, path=path)
+        torch.cuda.synchronize()
+        assert S.read_status(ws) == S.OK, (M, path)
+        assert_close(y, O.linear(x, q, s, 0, L.A, L.B, L.w_g, L.b_g)[0])

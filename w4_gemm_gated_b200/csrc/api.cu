@@ -96,19 +96,26 @@ struct WsLayout {
 
 static size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 
+// Every region that carries state between launches (header, flags,
+// tickets) sits at a fixed offset with capacity for the largest M, so one
+// workspace can serve any M, path and layer in any order; only the stateless
+// scratch after them (gated projection, K-split partials) grows with M.
+static constexpr int kMaxM = 65536;
+static constexpr int kFlagCap = kMaxM / 16 + 64;  // 16-token blocks (+ slack)
+
 static WsLayout ws_layout_uncached(const LayerView& L, int M_max) {
   WsLayout w = {};
   const int Mpad = ((M_max + 127) / 128) * 128;
-  const int RT = 32 * ((L.r / 16 + 2) / 2) + 16;  // >= decode (32*E2) and EC-kernel row strides
-  w.n_flags = Mpad / 16 + 64;
+  const int RT = 32 * ((128 / 16 + 2) / 2) + 16;  // row stride for the largest rank
+  w.n_flags = kFlagCap;
   size_t off = kWsHeaderBytes;
   w.hdr = 0;
   w.mflags = off;
-  off = up256(off + sizeof(int) * w.n_flags);
+  off = up256(off + sizeof(int) * kFlagCap);
   w.tickets = off;
-  off = up256(off + sizeof(int) * w.n_flags);
+  off = up256(off + sizeof(int) * kFlagCap);
   w.tcflags = off;
-  off = up256(off + sizeof(int) * w.n_flags);
+  off = up256(off + sizeof(int) * 4 * kFlagCap);
   w.t = off;
   off = up256(off + sizeof(float) * 16 * (size_t)RT);
   w.gt = off;

@@ -41,6 +41,7 @@ constexpr int TC_BM = 128;
 constexpr int TC_BN = 256;
 constexpr int TC_BK = 64;
 constexpr int TC_STAGES = 3;
+constexpr int TC_PREFETCH = 8;  // k-steps of L2 prefetch ahead of the TMA loads
 constexpr int TC_THREADS = 14 * 32;  // producer, mma, 4 epilogue, 8 dequant warps
 constexpr int TC_X_BYTES = TC_BM * TC_BK * 2;      // 16 KB
 constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;      // 32 KB
@@ -54,7 +55,7 @@ struct TcArgs {
   float* gate_out;
   int* mask_count;
   WsHeader* hdr;
-  int* mflags;        // per 128-token block: +1 per epilogue warp once its gt rows are out
+  int* mflags;        // [4 * Mb]: epoch + 1 once an epilogue warp's 32 gt rows are out
   __nv_bfloat16* gt;  // [Mb * 128][r]
   int M, K, N, r, group;
   float b_g, tau;
@@ -257,6 +258,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tma_load_2d(smem_u32(xd), &tm_x, &full[s], k * TC_BK, ti.mb * TC_BM);
             tma_load_2d(smem_u32(bd), &tm_agt, &full[s], k * TC_BK, 0);
           } else if (k < KT) {
+            // warm L2 a few k-steps ahead so the shallow shared-memory ring
+            // does not see the full HBM latency on every stage
+            if (k + TC_PREFETCH < KT) {
+              tma_prefetch_2d(&tm_x, (k + TC_PREFETCH) * TC_BK, ti.mb * TC_BM);
+              tma_prefetch_3d(&tm_w, 0, k + TC_PREFETCH, ti.nb * (TC_BN / 16));
+            }
+            if (k == 0)
+              for (int pk = 1; pk < TC_PREFETCH && pk < KT; ++pk) {
+                tma_prefetch_2d(&tm_x, pk * TC_BK, ti.mb * TC_BM);
+                tma_prefetch_3d(&tm_w, 0, pk, ti.nb * (TC_BN / 16));
+              }
             mbar_arrive_tx(&full[s], TC_X_BYTES + TC_P_BYTES);
             tma_load_2d(smem_u32(xd), &tm_x, &full[s], k * TC_BK, ti.mb * TC_BM);
             tma_load_3d(smem_u32(pd), &tm_w, &full[s], 0, k, ti.nb * (TC_BN / 16));
@@ -264,7 +276,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const int e = k - KT;
             if (e == 0) {
               // gated projection of this token block must be published
-              ok = wait_flag_eq(&a.mflags[ti.mb], 4 * (epoch + 1), a.hdr);
+              for (int qq = 0; qq < 4 && ok; ++qq) ok = wait_flag_eq(&a.mflags[4 * ti.mb + qq], epoch + 1, a.hdr);
               if (!ok) {
                 *abort_flag = 1;
                 break;
@@ -356,8 +368,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         __threadfence();
         tc_fence_before();
         __syncwarp();
-        // four epilogue warps per block: the block is ready at 4 * (epoch + 1)
-        if (lane == 0) atomicAdd(&a.mflags[ti.mb], 1);
+        // one flag per epilogue warp (32 token rows), tagged with this launch's epoch
+        if (lane == 0) st_release_gpu(&a.mflags[4 * ti.mb + q], epoch + 1);
       } else {
         const int n0 = ti.nb * TC_BN;
 #pragma unroll 1
