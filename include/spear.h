@@ -181,6 +181,27 @@ int spear_linear_forward_path(const spear_layer* layer, const uint16_t* x, int M
  * *device_status receives SPEAR_OK or the first device-side error code. */
 int spear_read_status(void* ws, int* device_status, void* stream);
 
+/* ---- allocation-free decode call ---------------------------------------------
+ * Not part of the method on the pages (they have no counterpart): an
+ * interface for callers that cannot allocate device memory where they run
+ * the layer -- code executing while another component owns the CUDA
+ * allocator (a serving engine's memory pool), token loops in which an
+ * allocation would synchronise the device, or plugin hosts that pass only
+ * input and output buffers.
+ * Same result as spear_linear_forward_path(..., SPEAR_PATH_DECODE, ...), but
+ * the scratch lives in a 16 KB device array inside the library instead of a
+ * caller workspace.  Limit: 1 <= M <= 16 (larger M returns
+ * SPEAR_ERR_UNSUPPORTED_SHAPE); every layer shape of the decode path.
+ * No device memory is allocated or freed.  The first call on a device looks
+ * up the array's device address (cudaGetSymbolAddress) and caches it, so
+ * make that first call before any stream capture.  Each call clears the
+ * array's launch header on `stream` before its kernel.  The array is shared
+ * by all calls on a device: calls whose executions may overlap on the GPU
+ * (other streams, unordered host threads) race and must not be issued. */
+int spear_linear_forward_decode_noalloc(const spear_layer* layer, const uint16_t* x, int M,
+                                        uint16_t* y, float* gate_out, int* mask_count,
+                                        void* stream);
+
 /* ---- a-7: dispatcher ----------------------------------------------------------
  * Phase-aware choice between the fused and the unfused EC path (SPEAR,
  * gist.science technical summary, section 2.2 A "Dispatch de fusion de noyau

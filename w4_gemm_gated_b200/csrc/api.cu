@@ -86,6 +86,9 @@ static int check_layer(const spear_layer* l, LayerView* out) {
   return SPEAR_OK;
 }
 
+int validate_layer(const spear_layer* layer, LayerView* out) { return check_layer(layer, out); }
+int device_sm_count() { return sm_count(); }
+
 // ---------------------------------------------------------------------------
 // workspace layout
 // ---------------------------------------------------------------------------

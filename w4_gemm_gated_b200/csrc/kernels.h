@@ -16,6 +16,12 @@ int set_cuda_error(const char* what, cudaError_t e);
 // Record a message as the thread's last error; returns `code`.
 int set_error(int code, const char* fmt, ...);
 
+struct LayerView;
+// Validate a public layer description (same checks as every layer call).
+int validate_layer(const struct spear_layer* layer, LayerView* out);
+// Multiprocessor count of the current device (cached).
+int device_sm_count();
+
 // A validated layer, with typed device pointers.
 struct LayerView {
   int K, N, group, r;

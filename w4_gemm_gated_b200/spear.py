@@ -74,6 +74,7 @@ EXPORTS = {
     "spear_linear_forward": (_i, ctypes.POINTER(LayerStruct), _vp, _i, _vp, _vp, _sz, _vp, _vp, _vp),
     "spear_linear_forward_path": (_i, ctypes.POINTER(LayerStruct), _vp, _i, _vp, _vp, _sz, _vp, _vp, _i, _vp),
     "spear_read_status": (_i, _vp, ctypes.POINTER(_i), _vp),
+    "spear_linear_forward_decode_noalloc": (_i, ctypes.POINTER(LayerStruct), _vp, _i, _vp, _vp, _vp, _vp),
     "spear_dispatch_choice": (_i, ctypes.POINTER(LayerStruct), _i),
     "spear_dispatch_tune": (_i, ctypes.POINTER(LayerStruct), ctypes.POINTER(_i), _i, _vp, _vp, _vp, _sz, _vp, _sz,
                             _i, ctypes.POINTER(_f), _vp),
@@ -240,6 +241,21 @@ def forward(layer: Layer, x: torch.Tensor, ws: torch.Tensor, y: torch.Tensor | N
     st = layer.struct()
     _check(F["spear_linear_forward_path"](ctypes.byref(st), _ptr(x), M, _ptr(y), _ptr(ws), ws.numel(),
                                           _ptr(gate_out), _ptr(mask_count), path, _stream(stream)))
+    return y
+
+
+def forward_decode_noalloc(layer: Layer, x: torch.Tensor, y: torch.Tensor | None = None,
+                           gate_out: torch.Tensor | None = None, mask_count: torch.Tensor | None = None,
+                           stream=None) -> torch.Tensor:
+    """Decode-path layer call for M <= 16 that allocates no device memory: its
+    scratch is a fixed array inside the library (shared by all calls on a
+    device, so calls must not overlap on the GPU)."""
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty((M, layer.N), dtype=torch.bfloat16, device=x.device)
+    st = layer.struct()
+    _check(F["spear_linear_forward_decode_noalloc"](ctypes.byref(st), _ptr(x), M, _ptr(y), _ptr(gate_out),
+                                                    _ptr(mask_count), _stream(stream)))
     return y
 
 
