@@ -55,7 +55,8 @@ constexpr int DEC_UNIT = 4096;    // bytes per unit
 constexpr int DEC_MAXSEG = 2;     // pairs one consumer may touch
 constexpr int DEC_MAXPAIRS = 64;  // pairs per cluster
 constexpr int DEC_MAXRING = 40;
-constexpr int DEC_MAXCL = 160;     // clusters described in the kernel parameters
+constexpr int DEC_MAXCL = 160;
+constexpr int DEC_PREWAIT = 8;     // units requested before the grid-dependency wait     // clusters described in the kernel parameters
 
 struct DecodeArgs {
   const __half* scales;
@@ -479,8 +480,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
   };
 
   // weights (and [A^T ; w_g]) do not depend on the previous kernel in the
-  // stream: the first ring-full is requested before the grid-dependency wait
+  // stream: a few units are requested before the grid-dependency wait; x goes
+  // right after the wait, ahead of the rest of the ring (so it does not queue
+  // behind megabytes of weight requests)
   const int first_batch = L.U < a.ring ? L.U : a.ring;
+  const int pre_batch = first_batch < DEC_PREWAIT ? first_batch : DEC_PREWAIT;
   if (warp == 0) {
     for (int s = lane; s < a.ring; s += 32) {
       mbar_init(&full[s], 1);
@@ -489,7 +493,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
     if (lane == 0) mbar_init(xbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncwarp();
-    for (int j = lane; j < first_batch; j += 32) {
+    for (int j = lane; j < pre_batch; j += 32) {
       int kind, c1, c2;
       job_of(j, kind, c1, c2);
       issue_job(j, kind, c1, c2);
@@ -522,6 +526,12 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
       mbar_arrive_tx(xbar, a.kt_part * MT * 128);
       for (int kt = 0; kt < a.kt_part; ++kt)
         tma_load_2d(smem_u32(xs + kt * MT * 128), &tm_x, xbar, q * kp + kt * 64, 0);
+    }
+    __syncwarp();
+    for (int j = pre_batch + lane; j < first_batch; j += 32) {
+      int kind, c1, c2;
+      job_of(j, kind, c1, c2);
+      issue_job(j, kind, c1, c2);
     }
     // remaining units: slot s is always refilled by lane s % 32, in issue
     // order, so no lane waits on a slot more than one phase ahead
