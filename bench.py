@@ -192,6 +192,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--profile-case", choices=["decode", "prefill"], default=None,
+                    help="run only --steps launches of one kernel on a small case (for ncu captures); "
+                         "prints no bench line")
+    ap.add_argument("--m", type=int, default=16, help="tokens of the --profile-case launch")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -202,6 +206,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.profile_case:
+        run_profile_case(args)
         return
 
     import torch
@@ -417,6 +424,37 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def run_profile_case(args):
+    """A few launches of one kernel for a profiler: the decode kernel on the
+    7B up-projection (K=4096, N=11008, r=64) or the tensor-core kernel on the
+    o-projection shape (K=N=4096, r=64), at --m tokens."""
+    import torch
+    from w4_gemm_gated_b200 import spear as S
+    from w4_gemm_gated_b200 import synth
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+    M = args.m
+    if args.profile_case == "decode":
+        L = synth.decode(16, force_outlier=True)
+        x = bf16(L.x[:M])
+        path = S.PATH_DECODE
+    else:
+        L = synth.prefill(M=M)
+        x = bf16(L.x)
+        path = S.PATH_FUSED
+    lay = S.prepare_layer(torch.from_numpy(L.W).cuda(), 0, bf16(L.A), bf16(L.B), bf16(L.w_g), L.b_g)
+    ws = S.make_workspace(lay, max(M, 16))
+    for _ in range(args.steps):
+        S.forward(lay, x, ws, path=path)
+    torch.cuda.synchronize()
+    st = S.read_status(ws)
+    print(json.dumps({"profile_case": args.profile_case, "M": M, "launches": args.steps, "status": st}))
+    if st != S.OK:
+        sys.exit(1)
 
 
 def bench_prefill(S, synth, dev, stream, bf16, tc_peak):

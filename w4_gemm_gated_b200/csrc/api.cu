@@ -120,7 +120,7 @@ static WsLayout ws_layout_uncached(const LayerView& L, int M_max) {
   w.tcflags = off;
   off = up256(off + sizeof(int) * 4 * kFlagCap);
   w.t = off;
-  off = up256(off + sizeof(float) * 16 * (size_t)RT);
+  off = up256(off + sizeof(float) * std::max<size_t>(16 * (size_t)RT, decode2_tt_bytes(128) / sizeof(float)));
   w.gt = off;
   off = up256(off + 2 * (size_t)Mpad * (L.r > 0 ? L.r : 1));
   w.part = off;
@@ -198,6 +198,8 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
   const int sms = sm_count();
   if (path == SPEAR_PATH_DECODE) {
     if (M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs M <= 16 (M=%d)", M);
+    if (!decode2_unsupported(M, L.K, L.N, L.r))
+      return launch_decode2(L, x, M, y, hdr, tbuf, gate_out, mask_count, false, st);
     DecodePlan p = plan_decode(M, L.K, L.N, L.r, L.group, sms);
     const char* why = check_decode_plan(p);
     if (why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", why);
@@ -209,7 +211,13 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
     L0.agt = nullptr;
     L0.bpt = nullptr;
     int rc;
-    if (M <= 16) {
+    if (M <= 16 && !decode2_unsupported(M, L.K, L.N, L.r)) {
+      rc = launch_decode2(L0, x, M, y, hdr, tbuf, L.r > 0 ? nullptr : gate_out, L.r > 0 ? nullptr : mask_count,
+                          false, st);
+      if (rc || L.r == 0) return rc;
+      // the separate EC launch: same kernel in EC-only mode, y += g (t . B) in place
+      return launch_decode2(L, x, M, y, hdr, tbuf, gate_out, mask_count, true, st);
+    } else if (M <= 16) {
       DecodePlan p = plan_decode(M, L.K, L.N, 0, L.group, sms);
       const char* why = check_decode_plan(p);
       if (why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", why);

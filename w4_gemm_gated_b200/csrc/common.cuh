@@ -23,7 +23,9 @@ struct WsHeader {
   int done_ctas;  // CTAs finished in the current launch
   int ec_done;    // EC row groups finalised in the current launch
   int ec_flag;    // == epoch + 1 once the gated EC projection of this launch is ready
-  int pad0[59];
+  int d2_epoch;   // decode path: launches completed (tags its EC projection words)
+  int gt_obs;     // decode path: CTAs that have read the complete EC projection
+  int pad0[57];
 };
 static_assert(sizeof(WsHeader) <= 256, "header must fit in 256 bytes");
 constexpr size_t kWsHeaderBytes = 256;
@@ -150,6 +152,35 @@ __device__ __forceinline__ uint32_t atom_add_dsmem_acqrel(uint32_t addr, uint32_
 
 __device__ __forceinline__ void fence_acq_rel_cluster() {
   asm volatile("fence.acq_rel.cluster;" ::: "memory");
+}
+
+// Non-blocking test of an mbarrier phase (local shared memory).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bulk copy global -> shared (16-byte aligned, size a multiple of 16), counted
+// on an mbarrier of this CTA.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// 16 bytes into the shared memory of another CTA of the cluster; completion
+// is counted (bytes) on an mbarrier of that CTA.  Both addresses come from mapa.
+__device__ __forceinline__ void st_async_f4(uint32_t remote, float4 v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   remote),
+               "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(remote_bar)
+               : "memory");
 }
 
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf(-z)); }

@@ -50,6 +50,14 @@ int launch_decode(const DecodePlan& p, const LayerView& L, const __nv_bfloat16* 
                   WsHeader* hdr, float* ws_t, __nv_bfloat16* ws_gt, float* gate_out, int* mask_count, bool ec_only,
                   cudaStream_t st);
 
+// ---- decode path for back-to-back launches (decode2.cu) ----
+// null if the kernel can run (M, K, N, r), else the reason
+const char* decode2_unsupported(int M, int K, int N, int r);
+// bytes of tagged EC projection words the kernel needs in the workspace
+size_t decode2_tt_bytes(int r);
+int launch_decode2(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, WsHeader* hdr, void* tt,
+                   float* gate_out, int* mask_count, bool ec_only, cudaStream_t st);
+
 // ---- standalone EC kernel (ec.cu): y += g * (x.A).B, in place ----
 struct EcPlan {
   int ksplit;   // K parts of the projection

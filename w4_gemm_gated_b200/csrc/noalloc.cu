@@ -22,13 +22,17 @@
 
 namespace spear {
 
-// Scratch capacity: header, projection rows [16 tokens][32 * E2 <= 176 fp32],
-// gated projection [16 tokens][r <= 128 bf16].
+// Scratch capacity: header, then either the tagged EC projection words of the
+// decode kernel ([9 EC strips][16 tokens][16 rows] x 8 bytes, r <= 128) or, for
+// shapes only the cluster split-K kernel runs, its projection rows [16 tokens]
+// [176 fp32] and gated projection [16][128 bf16].
 constexpr size_t kNoAllocHeader = kWsHeaderBytes;
+constexpr size_t kNoAllocEcp = 9 * 16 * 16 * 8;
 constexpr size_t kNoAllocT = 16 * 176 * sizeof(float);
 constexpr size_t kNoAllocGt = 16 * 128 * 2;
-constexpr size_t kNoAllocBytes = 16384;
+constexpr size_t kNoAllocBytes = 40960;
 static_assert(kNoAllocHeader + kNoAllocT + kNoAllocGt <= kNoAllocBytes, "scratch layout exceeds its array");
+static_assert(kNoAllocHeader + kNoAllocEcp <= kNoAllocBytes, "scratch layout exceeds its array");
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
 
@@ -69,17 +73,25 @@ extern "C" int spear_linear_forward_decode_noalloc(const spear_layer* layer, con
       (gate_out && (reinterpret_cast<uintptr_t>(gate_out) & 3)) ||
       (mask_count && (reinterpret_cast<uintptr_t>(mask_count) & 3)))
     return set_error(SPEAR_ERR_ALIGNMENT, "x and y must be 16-byte aligned");
-  const DecodePlan p = plan_decode(M, L.K, L.N, L.r, L.group, device_sm_count());
-  const char* why = check_decode_plan(p);
+  const bool v2 = decode2_unsupported(M, L.K, L.N, L.r) == nullptr;
+  if (v2 && decode2_tt_bytes(L.r) > kNoAllocEcp)
+    return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "EC projection scratch exceeds the allocation-free array");
+  const DecodePlan p = v2 ? DecodePlan{} : plan_decode(M, L.K, L.N, L.r, L.group, device_sm_count());
+  const char* why = v2 ? nullptr : check_decode_plan(p);
   if (why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", why);
   uint8_t* scratch = nullptr;
   rc = noalloc_scratch_ptr(&scratch);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // the launch header (epoch, arrival counters, flags) must start at zero
-  cudaError_t e = cudaMemsetAsync(scratch, 0, kNoAllocHeader, st);
+  // the launch header (epoch, arrival counters, flags) and the tagged EC
+  // projection words (their tags are checked against the header's epoch) must
+  // start at zero
+  cudaError_t e = cudaMemsetAsync(scratch, 0, kNoAllocHeader + (v2 ? kNoAllocEcp : 0), st);
   if (e != cudaSuccess) return set_cuda_error("scratch header clear", e);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(scratch);
+  if (v2)
+    return launch_decode2(L, reinterpret_cast<const __nv_bfloat16*>(x), M, reinterpret_cast<__nv_bfloat16*>(y), hdr,
+                          scratch + kNoAllocHeader, gate_out, mask_count, false, st);
   float* tbuf = reinterpret_cast<float*>(scratch + kNoAllocHeader);
   __nv_bfloat16* gt = reinterpret_cast<__nv_bfloat16*>(scratch + kNoAllocHeader + kNoAllocT);
   return launch_decode(p, L, reinterpret_cast<const __nv_bfloat16*>(x), M, reinterpret_cast<__nv_bfloat16*>(y), hdr,
