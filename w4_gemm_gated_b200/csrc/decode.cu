@@ -421,7 +421,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
   constexpr int NT = MT / 8;
   constexpr int NF4 = 2 * NT;  // float4 fragments per lane per slot
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  // 1024-byte aligned base, derived from the shared array itself so that the
+  // compiler keeps every access in the shared window (ld/st.shared)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* ring = smem;                                       // [ring][4 KB]
   uint8_t* xs = ring + (size_t)a.ring * DEC_UNIT;             // [kt_part][MT x 128 B], swizzled
   float4* slots = reinterpret_cast<float4*>(xs + (size_t)a.kt_part * MT * 128);

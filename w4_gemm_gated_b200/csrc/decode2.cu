@@ -53,7 +53,9 @@ constexpr int D2_NWC = 4;                       // consumer warps (one per SM su
 constexpr int D2_THREADS = (D2_NWC + 2) * 32;   // + one producer and one reducer warp
 constexpr int D2_SLOT = 8192;                   // ring slot bytes
 constexpr int D2_MAXSLOT = 16;
-constexpr int D2_NBUF = 4;                      // partial-sum buffers (jobs in flight per CTA)
+// partial-sum buffers (jobs in flight per CTA) and weight strips per job
+__host__ __device__ constexpr int d2_nbuf(int MT) { return 4; }
+__host__ __device__ constexpr int d2_bj(int MT) { return MT > 0 ? 1 : 1; }
 constexpr int D2_MAXCL = 160;                   // clusters described in the kernel parameters
 constexpr int D2_MAXOWN = 16;                   // strips one CTA finishes per launch
 constexpr int D2_KTW_MAX = 8;                   // warp slice (k-tiles): KTW * NT * 8 activation registers
@@ -98,7 +100,7 @@ __host__ __device__ __forceinline__ D2Smem d2_smem(int MT, int nslot, int CS, in
   s.ring = off;
   off += nslot * D2_SLOT;
   s.red = off;
-  off += D2_NBUF * D2_NWC * NT * 512;
+  off += d2_nbuf(MT) * D2_NWC * d2_bj(MT) * NT * 512;
   s.recv = off;
   off += CS > 1 ? own_cap * (CS - 1) * NT * 512 : 0;
   s.park = off;
@@ -114,7 +116,7 @@ __host__ __device__ __forceinline__ D2Smem d2_smem(int MT, int nslot, int CS, in
   s.stage = off;
   off += MT * 32;
   s.bars = off;
-  off += (2 * nslot + 2 * D2_NBUF + own_cap + 2) * 8;
+  off += (2 * nslot + 2 * d2_nbuf(MT) + own_cap + 2) * 8;
   s.total = off + 1024;  // base alignment slack
   return s;
 }
@@ -153,7 +155,39 @@ __device__ __forceinline__ bool d2_wait_idle(uint64_t* bar, uint32_t parity, vol
   return true;
 }
 __device__ __forceinline__ bool d2_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, WsHeader* h) {
-  return d2_wait_idle(bar, parity, abort_flag, h, 1000u, [] {});
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (int it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63) == 0) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > kWaitCycles) {
+        report_status(h, SPEAR_ERR_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait for warps that must not take issue slots from the consumer
+// warps: a non-blocking test, then sleeps of growing length (up to max_ns).
+__device__ __forceinline__ bool d2_wait_polite(uint64_t* bar, uint32_t parity, volatile int* abort_flag, WsHeader* h,
+                                               uint32_t max_ns) {
+  if (mbar_test(bar, parity)) return true;
+  const long long t0 = clock64();
+  uint32_t ns = 32;
+  while (true) {
+    __nanosleep(ns);
+    if (mbar_test(bar, parity)) return true;
+    ns = ns * 2 < max_ns ? ns * 2 : max_ns;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      report_status(h, SPEAR_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
 }
 
 // Swizzled 128-byte-row tile (TMA SWIZZLE_128B): 16-byte chunk ch of row r.
@@ -323,13 +357,16 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
     decode2_kernel(const __grid_constant__ D2Args a, const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ CUtensorMap tm_agt, const __grid_constant__ CUtensorMap tm_bp) {
   constexpr int NT = D2T<MT>::NT, ACCS = D2T<MT>::ACCS;
+  constexpr int NBUF = d2_nbuf(MT), BJ = d2_bj(MT);
   constexpr int WPU = d2_wpu(KTW), ECU = d2_ecu(KTW) < KTW ? d2_ecu(KTW) : KTW;
   constexpr int UPJ = D2_NWC / WPU;  // units per job and pass
   constexpr int R = KTW / ECU;       // passes over an EC strip (ECU tiles per warp each)
   constexpr unsigned FULL = 0xffffffffu;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int s_abort;
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  // 1024-byte aligned base, derived from the shared array itself so that the
+  // compiler keeps every access in the shared window (ld/st.shared)
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const D2Smem SL = d2_smem(MT, a.nslot, a.CS, a.own_cap, a.r, a.ES);
   uint8_t* ring = sm + SL.ring;
   float4* red = reinterpret_cast<float4*>(sm + SL.red);
@@ -343,8 +380,8 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + SL.bars);
   uint64_t* empty = full + a.nslot;
   uint64_t* redfull = empty + a.nslot;
-  uint64_t* redempty = redfull + D2_NBUF;
-  uint64_t* recvbar = redempty + D2_NBUF;
+  uint64_t* redempty = redfull + NBUF;
+  uint64_t* recvbar = redempty + NBUF;
   uint64_t* epibar = recvbar + a.own_cap;
   uint64_t* tsbar = epibar + 1;  // completion of the reducer's cp.async fetches (one arrival per lane)
 
@@ -352,7 +389,11 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
   const int q = a.CS > 1 ? (int)cluster_rank() : 0;
   const short4 ct = a.cl_tab[blockIdx.x / a.CS];
   const int ec_lo = ct.x, n_ec = ct.y, w_lo = ct.z, n_w = ct.w;
-  const int n_jobs = n_ec + n_w;
+  const int n_jobs = n_ec + n_w;                           // items: EC strips, then weight strips
+  // jobs (units of synchronisation): one per EC strip, then weight strips in groups of BJ
+  const int n_jb = n_ec + (n_w + BJ - 1) / BJ;
+  auto job_first = [&](int j) { return j < n_ec ? j : n_ec + (j - n_ec) * BJ; };
+  auto job_len = [&](int j) { return j < n_ec ? 1 : min(BJ, n_jobs - (n_ec + (j - n_ec) * BJ)); };
   const int ecU = n_ec * R * UPJ;                          // EC units come first
   const int U = ecU + (a.ec_only ? 0 : n_w * UPJ);
   const bool has_ec = a.ES > 0;
@@ -384,7 +425,7 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], WPU);
     }
-    if (lane < D2_NBUF) {
+    if (lane < NBUF) {
       mbar_init(&redfull[lane], D2_NWC);
       mbar_init(&redempty[lane], 1);
     }
@@ -447,11 +488,16 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     // units in order: wait (sleeping) for the slot to drain, lane 0 refills it
+    int slot = 0;
+    uint32_t round = 1;  // u / nslot
     for (int u = a.nslot; u < U; ++u) {
-      const int slot = u % a.nslot;
-      if (!__all_sync(FULL, d2_wait(&empty[slot], ((u / a.nslot) & 1) ^ 1, abortp, a.hdr))) break;
+      if (!__all_sync(FULL, d2_wait_polite(&empty[slot], (round & 1) ^ 1, abortp, a.hdr, 256u))) break;
       if (lane == 0) issue(slot, u);
       __syncwarp();
+      if (++slot == a.nslot) {
+        slot = 0;
+        ++round;
+      }
     }
     if (a.CS > 1) asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
   } else if (warp <= D2_NWC) {
@@ -498,10 +544,21 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
       }
     }
     if (a.CS > 1) asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
-    const int n_part = a.ec_only ? n_ec : n_jobs;  // jobs with weight or EC partials
     bool ok = true;
-    for (int i = 0; i < n_part && ok; ++i) {
-      float acc[NT][4];
+    // this warp's units are g, g + UPJ, g + 2 UPJ, ...: ring slot and phase of the next one
+    int cslot = g;
+    uint32_t cphase = 0;
+    auto next_unit = [&](int& slot, uint32_t& phase) {
+      slot = cslot;
+      phase = cphase;
+      cslot += UPJ;
+      if (cslot >= a.nslot) {
+        cslot -= a.nslot;
+        cphase ^= 1u;
+      }
+    };
+    // one item (an EC strip or a weight strip) of this warp's slice into acc
+    auto compute_item = [&](int i, float (&acc)[NT][4]) -> bool {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
       if (i < n_ec) {
@@ -511,9 +568,9 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
 #pragma unroll
         for (int kt = 0; kt < KTW; ++kt) {
           if (kt % ECU == 0) {
-            const int u = (i * R + kt / ECU) * UPJ + g;
-            slot = u % a.nslot;
-            ok = ok && __all_sync(FULL, d2_wait(&full[slot], (u / a.nslot) & 1, abortp, a.hdr));
+            uint32_t phase;
+            next_unit(slot, phase);
+            ok = ok && __all_sync(FULL, d2_wait(&full[slot], phase, abortp, a.hdr));
             src = ring + (size_t)slot * D2_SLOT + wi * ECU * 2048;
           }
           if (ok) d2_ec_tile<NT>(src + (kt % ECU) * 2048, xf[kt], lane, acc);
@@ -522,10 +579,12 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
             if (lane == 0) mbar_arrive(&empty[slot]);
           }
         }
-        if (!ok) break;
+        if (!ok) return false;
       } else {
-        const int u = ecU + (i - n_ec) * UPJ + g, slot = u % a.nslot;
-        if (!__all_sync(FULL, d2_wait(&full[slot], (u / a.nslot) & 1, abortp, a.hdr))) break;
+        int slot;
+        uint32_t phase;
+        next_unit(slot, phase);
+        if (!__all_sync(FULL, d2_wait(&full[slot], phase, abortp, a.hdr))) return false;
         const uint8_t* src = ring + (size_t)slot * D2_SLOT + wi * KTW * 512 + lane * 16;
         if (GROUP) {
           const int p = w_lo + (i - n_ec);
@@ -591,12 +650,27 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
       }
-      // the partial goes to the reducer warp through buffer b
-      const int b = i % D2_NBUF, k = i / D2_NBUF;
+      return true;
+    };
+    const int n_jp = a.ec_only ? n_ec : n_jb;  // jobs with weight or EC partials
+    for (int j = 0; j < n_jp && ok; ++j) {
+      const int t0 = job_first(j), nb = job_len(j);
+      float accb[BJ][NT][4];
+#pragma unroll
+      for (int sb = 0; sb < BJ; ++sb)
+        if (sb < nb && ok) ok = compute_item(t0 + sb, accb[sb]);
+      if (!ok) break;
+      // the partials go to the reducer warp through buffer b
+      const int b = j % NBUF, k = j / NBUF;
       if (!__all_sync(FULL, d2_wait(&redempty[b], (k & 1) ^ 1, abortp, a.hdr))) break;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        red[((b * D2_NWC + w) * NT + nt) * 32 + lane] = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
+      for (int sb = 0; sb < BJ; ++sb)
+        if (sb < nb) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            red[(((b * D2_NWC + w) * BJ + sb) * NT + nt) * 32 + lane] =
+                make_float4(accb[sb][nt][0], accb[sb][nt][1], accb[sb][nt][2], accb[sb][nt][3]);
+        }
       __syncwarp();
       if (lane == 0) mbar_arrive(&redfull[b]);
     }
@@ -655,8 +729,11 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
     auto rwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       if (__all_sync(FULL, mbar_test(bar, parity))) return true;
       const long long t0 = clock64();
+      uint32_t ns = 32;
       while (true) {
-        const bool d = mbar_try_wait_sleep(bar, parity, 300u);
+        __nanosleep(ns);
+        ns = ns < 256 ? ns * 2 : 256;
+        const bool d = mbar_test(bar, parity);
         if (__all_sync(FULL, d)) return true;
         int stop = 0;
         if (lane == 0) {
@@ -768,56 +845,63 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
       }
     };
 
-    for (int i = 0; i < n_jobs && ok; ++i) {
+    for (int j = 0; j < n_jb && ok; ++j) {
       if (gst < 3) gt_step();
-      const bool has_part = !(a.ec_only && i >= n_ec);
-      const int owner = i % a.CS, o = i / a.CS;
-      const bool mine = owner == q;
-      float tot[NT][4];
+      const int t0 = job_first(j), nb = job_len(j);
+      const bool has_part = !(a.ec_only && j >= n_ec);
+      const int b = j % NBUF, k = j / NBUF;
+      if (has_part && !rwait(&redfull[b], k & 1)) {
+        ok = false;
+        break;
+      }
+      for (int sb = 0; sb < nb; ++sb) {
+        const int i = t0 + sb;  // item
+        const int owner = i % a.CS, o = i / a.CS;
+        const bool mine = owner == q;
+        float tot[NT][4];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) tot[nt][0] = tot[nt][1] = tot[nt][2] = tot[nt][3] = 0.f;
-      if (has_part) {
-        const int b = i % D2_NBUF, k = i / D2_NBUF;
-        if (!rwait(&redfull[b], k & 1)) {
-          ok = false;
-          break;
-        }
-        for (int w2 = 0; w2 < D2_NWC; ++w2)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const float4 v = red[((b * D2_NWC + w2) * NT + nt) * 32 + lane];
-            tot[nt][0] += v.x;
-            tot[nt][1] += v.y;
-            tot[nt][2] += v.z;
-            tot[nt][3] += v.w;
-          }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&redempty[b]);
-        if (a.CS > 1) {
-          if (!mine) {
-            // this CTA's partial to the owner, which adds the ranks in order
-            const int sidx = q - (q > owner ? 1 : 0);
-            const uint32_t rbar = map_rank(smem_u32(&recvbar[o]), owner);
+        for (int nt = 0; nt < NT; ++nt) tot[nt][0] = tot[nt][1] = tot[nt][2] = tot[nt][3] = 0.f;
+        if (has_part) {
+          for (int w2 = 0; w2 < D2_NWC; ++w2)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              const uint32_t dst =
-                  map_rank(smem_u32(recv + ((o * (a.CS - 1) + sidx) * NT + nt) * 32 + lane), owner);
-              st_async_f4(dst, make_float4(tot[nt][0], tot[nt][1], tot[nt][2], tot[nt][3]), rbar);
+              const float4 v = red[(((b * D2_NWC + w2) * BJ + sb) * NT + nt) * 32 + lane];
+              tot[nt][0] += v.x;
+              tot[nt][1] += v.y;
+              tot[nt][2] += v.z;
+              tot[nt][3] += v.w;
             }
-          } else {
+          if (a.CS > 1) {
+            if (!mine) {
+              // this CTA's partial to the owner, which adds the ranks in order
+              const int sidx = q - (q > owner ? 1 : 0);
+              const uint32_t rbar = map_rank(smem_u32(&recvbar[o]), owner);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-              park[(o * NT + nt) * 32 + lane] = make_float4(tot[nt][0], tot[nt][1], tot[nt][2], tot[nt][3]);
-            __syncwarp();
-            pending |= 1u << o;
+              for (int nt = 0; nt < NT; ++nt) {
+                const uint32_t dst =
+                    map_rank(smem_u32(recv + ((o * (a.CS - 1) + sidx) * NT + nt) * 32 + lane), owner);
+                st_async_f4(dst, make_float4(tot[nt][0], tot[nt][1], tot[nt][2], tot[nt][3]), rbar);
+              }
+            } else {
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                park[(o * NT + nt) * 32 + lane] = make_float4(tot[nt][0], tot[nt][1], tot[nt][2], tot[nt][3]);
+              __syncwarp();
+              pending |= 1u << o;
+            }
+            continue;
           }
-          finish_pending(false);
+        } else if (!mine) {
           continue;
         }
-      } else if (!mine) {
-        continue;
+        finalize(i, tot);
+        if (!ok) break;
       }
-      finalize(i, tot);
+      if (has_part) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&redempty[b]);
+      }
+      if (a.CS > 1) finish_pending(false);
     }
     if (ok) finish_pending(true);
     if (ok && has_ec) {
@@ -840,7 +924,7 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
           ok = false;
           break;
         }
-        __nanosleep(100);
+        __nanosleep(256);
       }
       flush_parked();
       if (lane == 0 && obs_prev == a.G - 1) {

@@ -192,7 +192,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_agt,
               const __grid_constant__ CUtensorMap tm_bpt, const __grid_constant__ CUtensorMap tm_gt) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  // 1024-byte aligned base, derived from the shared array itself so that the
+  // compiler keeps every access in the shared window (ld/st.shared)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* xs = smem;                                        // [STAGES][16 KB]
   uint8_t* bs = smem + TC_STAGES * TC_X_BYTES;               // [STAGES][32 KB]
   uint8_t* ps = bs + TC_STAGES * TC_B_BYTES;                 // [STAGES][8 KB]
