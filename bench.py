@@ -154,6 +154,21 @@ def time_oracle(target_s: float = 15.0, n_cols: int = 1376):
                       f"{el:.1f} s, scaled to the full layer by column fraction"}
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's elapsed time (every rank calls this, in the same order)."""
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_step_per_rank: float, steps: int, world: int, max_ms: float) -> float:
+    """Units processed by all ranks (replicas: every rank runs the same step) per second."""
+    return units_per_step_per_rank * steps * world / (max_ms * 1e-3)
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -196,6 +211,10 @@ def main():
                     help="run only --steps launches of one kernel on a small case (for ncu captures); "
                          "prints no bench line")
     ap.add_argument("--m", type=int, default=16, help="tokens of the --profile-case launch")
+    ap.add_argument("--sweep", action="store_true",
+                    help="dispatch sweep (M x (K, N) x r x scale kind): time every path, check the dispatcher")
+    ap.add_argument("--stack", action="store_true",
+                    help="32-layer decoder stack of W4 linears (ECs on layers 0, 1, 30, 31) at M=256")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -209,6 +228,12 @@ def main():
         return
     if args.profile_case:
         run_profile_case(args)
+        return
+    if args.sweep:
+        run_sweep(args)
+        return
+    if args.stack:
+        run_stack(args)
         return
 
     import torch
@@ -296,11 +321,7 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    el_ms = e0.elapsed_time(e1)
-    t = torch.tensor([el_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    el_ms = float(t.item())
+    el_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     assert S.read_status(ws, stream=stream) == S.OK
 
     # The timed region holds nothing but decode-kernel launches (3 per step),
@@ -328,7 +349,7 @@ def main():
         mean_us[M] = m0.elapsed_time(m1) * 1e3 / (4 * 3 * ncopy)
 
     tokens_per_step = sum(MS)
-    value = tokens_per_step * args.steps * world / (el_ms * 1e-3)
+    value = whole_job_rate(tokens_per_step, args.steps, world, el_ms)
 
     # ---- end to end through the public API: pinned host x in, host y out ----
     hx = {M: xs[M].cpu().pin_memory() for M in MS}
@@ -353,11 +374,7 @@ def main():
             e2e_step(i)
         a1.record(stream)
         a1.synchronize()
-    e2e_ms = a0.elapsed_time(a1)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = tokens_per_step * e2e_steps * world / (float(te.item()) * 1e-3)
+    e2e_value = whole_job_rate(tokens_per_step, e2e_steps, world, max_over_ranks(a0.elapsed_time(a1), world, dev))
 
     # ---- EC overhead: same kernel with the EC disabled ----
     plain = [S.Layer(K_, N_, 0, 0, lay.w_packed, lay.scales, None, None, 0.0) for lay in layers]
@@ -424,6 +441,189 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+SWEEP_MS = (1, 8, 32, 128, 512, 2048, 8192)
+SWEEP_KN = ((4096, 4096), (4096, 14336), (14336, 4096))
+SWEEP_R = (32, 128)
+
+
+def run_sweep(args):
+    """Dispatch sweep: every (K, N, r, scale kind) layer is tuned over the M list
+    (spear_dispatch_tune: cold L2, CUDA events, median), then every eligible
+    path is re-timed independently and the table's choice is checked against
+    the fastest (within 5 %, or 2 us at small sizes)."""
+    import torch
+    from w4_gemm_gated_b200 import spear as S
+    from w4_gemm_gated_b200 import synth
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def median_us(layer, x, y, ws, path, reps):
+        ts = []
+        for i in range(reps + 3):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            S.forward(layer, x, ws, y=y, path=path, stream=stream)
+            b.record(stream)
+            b.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b) * 1e3)
+        return float(np.median(ts))
+
+    names = {S.PATH_DECODE: "decode", S.PATH_FUSED: "fused", S.PATH_UNFUSED: "unfused"}
+    points, good = [], 0
+    S.dispatch_clear()
+    t_start = time.perf_counter()
+    for K, N in SWEEP_KN:
+        L = synth.sweep_point(max(SWEEP_MS), K, N, 128)
+        W = torch.from_numpy(L.W).cuda()
+        x_all = bf16(L.x)
+        for r in SWEEP_R:
+            A, B, w_g = bf16(L.A[:, :r]), bf16(L.B[:r]), bf16(L.w_g)
+            for group in (0, 128):
+                layer = S.prepare_layer(W, group, A, B, w_g, L.b_g)
+                ws = S.make_workspace(layer, max(SWEEP_MS))
+                y_all = torch.empty((max(SWEEP_MS), N), dtype=torch.bfloat16, device="cuda")
+                S.dispatch_tune(layer, list(SWEEP_MS), x_all, y_all, ws, flush=flush, reps=10)
+                for M in SWEEP_MS:
+                    paths = [S.PATH_FUSED, S.PATH_UNFUSED] + ([S.PATH_DECODE] if M <= 16 else [])
+                    x = x_all[:M].contiguous()
+                    t = {p: median_us(layer, x, y_all[:M], ws, p, 10) for p in paths}
+                    choice = S.dispatch_choice(layer, M)
+                    best = min(t.values())
+                    ok = t[choice] <= max(1.05 * best, best + 2.0)
+                    good += ok
+                    fl = 2.0 * M * K * N + 2.0 * M * K * (r + 1) + 2.0 * M * r * N
+                    points.append({"M": M, "K": K, "N": N, "r": r, "group": group,
+                                   "us": {names[p]: round(v, 2) for p, v in t.items()},
+                                   "choice": names[choice], "choice_ok": bool(ok),
+                                   "tflops_best": round(fl / (best * 1e-6) / 1e12, 2)})
+                if S.read_status(ws) != S.OK:
+                    raise SystemExit("device status not OK during the sweep")
+                del layer, ws, y_all
+        del W, x_all
+    S.dispatch_clear()
+    print(json.dumps({"sweep": "dispatch (M x (K,N) x r x scale kind)", "points": len(points),
+                      "dispatcher_within_5pct": good, "seconds": round(time.perf_counter() - t_start, 1),
+                      "timing": "median of 10 launches, L2 flushed (256 MB write) before each",
+                      "table": points}))
+
+
+STACK_SHAPES = ((4096, 4096), (4096, 4096), (4096, 4096), (4096, 4096),  # q, k, v, o
+                (4096, 11008), (4096, 11008), (11008, 4096))              # gate, up, down
+STACK_EC_LAYERS = (0, 1, 30, 31)
+
+
+def stack_glue(S, layers, x, ws, eps=1e-6, n_layers=32):
+    """One pass of the synthetic decoder stack through the W4 (+EC) linears.
+    Per layer: h = RMSNorm(x); q, k, v = Wq h, Wk h, Wv h; x = x + Wo v (the
+    attention mixing is replaced by v); h2 = RMSNorm(x); x = x + Wd(silu(Wg h2) * Wu h2).
+    The glue between linears is plain tensor arithmetic (fp32, bf16 activations)."""
+    import torch
+
+    def rms(t):
+        tf = t.float()
+        return (tf * torch.rsqrt(tf.pow(2).mean(-1, keepdim=True) + eps)).to(torch.bfloat16)
+
+    for l in range(n_layers):
+        Lq, Lk, Lv, Lo, Lg, Lu, Ld = layers[l]
+        h = rms(x)
+        S.forward(Lq, h, ws)
+        S.forward(Lk, h, ws)
+        v = S.forward(Lv, h, ws)
+        x = (x.float() + S.forward(Lo, v, ws).float()).to(torch.bfloat16)
+        h2 = rms(x)
+        gte = S.forward(Lg, h2, ws).float()
+        up = S.forward(Lu, h2, ws).float()
+        act = (gte * torch.sigmoid(gte) * up).to(torch.bfloat16)
+        x = (x.float() + S.forward(Ld, act, ws).float()).to(torch.bfloat16)
+    return x
+
+
+def run_stack(args):
+    """Config 4: 32 decoder layers x 7 per-channel W4 linears, ECs (r=64) on all
+    linears of layers 0, 1, 30, 31, M=256 tokens pushed through all 224 linears.
+    Weights are drawn on the device (seeded per projection) and quantised and
+    packed by the library.  Reports the time of the linears alone and of the
+    whole stack with the glue."""
+    import torch
+    from w4_gemm_gated_b200 import spear as S
+    from w4_gemm_gated_b200 import synth
+
+    M, R = 256, 64
+    dev = torch.device("cuda")
+    layers, packed_bytes, ec_params = [], 0, 0
+    t0 = time.perf_counter()
+    for l in range(32):
+        row = []
+        for proj, (K, N) in enumerate(STACK_SHAPES):
+            g = torch.Generator(device=dev).manual_seed(synth.stack_layer_seed(0, l, proj))
+            W = torch.randn((K, N), generator=g, device=dev, dtype=torch.float32) * 0.02
+            if l in STACK_EC_LAYERS:
+                A = (torch.randn((K, R), generator=g, device=dev) * 0.01).to(torch.bfloat16)
+                B = (torch.randn((R, N), generator=g, device=dev) * 0.01).to(torch.bfloat16)
+                w_g = (torch.randn(K, generator=g, device=dev) / np.sqrt(K)).to(torch.bfloat16)
+                lay = S.prepare_layer(W, 0, A, B, w_g, -1.0)
+                ec_params += K * R + R * N + K
+            else:
+                lay = S.prepare_layer(W, 0, None, None, None, 0.0)
+            packed_bytes += K * N // 2
+            row.append(lay)
+            del W
+        layers.append(row)
+    prep_s = time.perf_counter() - t0
+    # one zeroed workspace large enough for every linear of the stack
+    ws = torch.zeros(max(S.workspace_bytes(lay, M) for row in layers for lay in row), dtype=torch.uint8, device=dev)
+    x0 = torch.randn((M, 4096), generator=torch.Generator(device=dev).manual_seed(7), device=dev).to(torch.bfloat16)
+    stream = torch.cuda.current_stream()
+
+    # the linears alone, inputs prepared once per shape
+    xs = {4096: x0, 11008: torch.randn((M, 11008), device=dev).to(torch.bfloat16)}
+    for _ in range(2):
+        for row in layers:
+            for lay in row:
+                S.forward(lay, xs[lay.K], ws)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(1, min(args.steps, 5))
+    a.record(stream)
+    for _ in range(reps):
+        for row in layers:
+            for lay in row:
+                S.forward(lay, xs[lay.K], ws)
+    b.record(stream)
+    b.synchronize()
+    lin_ms = a.elapsed_time(b) / reps
+
+    # the whole stack with the glue
+    for _ in range(2):
+        out = stack_glue(S, layers, x0, ws)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(reps):
+        out = stack_glue(S, layers, x0, ws)
+    b.record(stream)
+    b.synchronize()
+    e2e_ms = a.elapsed_time(b) / reps
+    assert S.read_status(ws) == S.OK
+    finite = bool(torch.isfinite(out.float()).all().item())
+    flops = sum(2.0 * M * K * N for (K, N) in STACK_SHAPES) * 32 + \
+        len(STACK_EC_LAYERS) * sum(2.0 * M * K * (R + 1) + 2.0 * M * R * N for (K, N) in STACK_SHAPES)
+    print(json.dumps({
+        "stack": "32 decoder layers x 7 W4 linears, ECs r=64 on layers 0,1,30,31", "M": M,
+        "linears_ms": lin_ms, "stack_ms": e2e_ms, "tokens_per_s": M / (e2e_ms * 1e-3),
+        "linears_tflops": flops / (lin_ms * 1e-3) / 1e12,
+        "packed_weight_bytes": packed_bytes, "ec_params": ec_params,
+        "ec_params_fraction_of_packed_bytes": ec_params / packed_bytes,
+        "ec_bytes_fraction_of_packed_bytes": 2 * ec_params / packed_bytes,
+        "output_finite": finite, "prep_seconds": round(prep_s, 1),
+        "timing": f"mean of {reps} passes, weights 3.24 GB (no L2 reuse across passes)"}))
 
 
 def run_profile_case(args):
