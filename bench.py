@@ -154,6 +154,29 @@ def time_oracle(target_s: float = 15.0, n_cols: int = 1376):
                       f"{el:.1f} s, scaled to the full layer by column fraction"}
 
 
+# DRAM bytes per decode launch from the ncu captures summarised in profiles/
+# (dram__bytes_read.sum + dram__bytes_write.sum, one launch at M = 1 and at M = 16),
+# valid only while the decode kernel sources are the ones captured.
+DECODE_TRAFFIC = {"sources_sha1": "79682818ddf8a7f9d15c7a047b085986282a8eaa",
+                  "bytes_per_launch": {1: 24614912, 16: 24743936}}
+DECODE_SOURCES = ("w4_gemm_gated_b200/csrc/decode2.cu", "w4_gemm_gated_b200/csrc/common.cuh",
+                  "w4_gemm_gated_b200/csrc/tma.cuh")
+
+
+def decode_traffic_per_step():
+    """DRAM bytes of one step (M = 1, 4, 16) from the captures, or None if the
+    kernel changed since (M = 4 runs the M = 1 instantiation; its x adds 24 KB)."""
+    import hashlib
+    h = hashlib.sha1()
+    for f in DECODE_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != DECODE_TRAFFIC["sources_sha1"]:
+        return None
+    b = DECODE_TRAFFIC["bytes_per_launch"]
+    return b[1] + (b[1] + 2 * 3 * 4096) + b[16]
+
+
 def max_over_ranks(ms: float, world: int, device) -> float:
     """The slowest rank's elapsed time (every rank calls this, in the same order)."""
     import torch
@@ -419,7 +442,8 @@ def main():
                    "timing": f"CUDA-graph replay of {chunk}-step chunks (launches overlap through programmatic "
                              f"dependent launch), events on the launching stream"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None,
+                     "frac": achieved / hbm_peak, "traffic": decode_traffic_per_step(),
+                     "traffic_unit": "DRAM bytes per step (3 launches), ncu capture in profiles/",
                      "kernel": "decode_kernel (fused W4 GEMV + gated EC)",
                      "per_launch_us": mean_us,
                      "achieved_from": "algorithmic bytes of a step / timed step time (3 decode launches)",
