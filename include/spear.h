@@ -226,11 +226,37 @@ int spear_dispatch_tune(const spear_layer* layer, const int* Ms, int nM,
 
 /* Set one table entry by hand (path is a SPEAR_PATH_* other than AUTO). */
 int spear_dispatch_set(int K, int N, int r, int group, int M, int path);
+/* Set one table entry with its measured time in microseconds (us >= 0).
+ * Entries made by spear_dispatch_set carry no time; spear_dispatch_tune
+ * records the median of the path it picks. */
+int spear_dispatch_set_time(int K, int N, int r, int group, int M, int path, float us);
+/* Measured time (microseconds) of the table's path for this layer at M's
+ * bucket.  SPEAR_ERR_INVALID_ARG if that entry has no time. */
+int spear_dispatch_time_us(const spear_layer* layer, int M, float* us);
 /* Forget every table entry. */
 void spear_dispatch_clear(void);
-/* Save / load the table as text (host file path). */
+/* Save / load the table as text (host file path).  Lines are
+ * "K N r group M_bucket path time_us"; a line without the time loads as
+ * not measured. */
 int spear_dispatch_save(const char* path);
 int spear_dispatch_load(const char* path);
+
+/* ---- SLO-constrained prefill chunk size --------------------------------------
+ * SPEAR, gist.science technical summary, section 2.2 C ("Ordonnancement par
+ * blocs conscient de l'EC et contraint par les SLO"): pick the largest prefill
+ * chunk whose predicted step time meets the inter-token latency SLO, from the
+ * precomputed kernel latency table.
+ * A step pushes decode_tokens + chunk tokens through each of layers[0..n_layers)
+ * (host array of layer pointers, EC on some of them or not).  Its predicted
+ * time is step_overhead_us plus, per layer, the table's measured time at the
+ * step's M bucket.  Candidates are chunks[0..n_chunks) (>= 0, any order).
+ * On success *chunk_out is the largest candidate whose prediction is
+ * <= slo_us (0 if none is), and *predicted_us (optional) its prediction (-1
+ * if none).  SPEAR_ERR_INVALID_ARG if a needed table entry has no measured
+ * time (tune those M buckets first).  Host only; no GPU work. */
+int spear_slo_chunk(const spear_layer* const* layers, int n_layers, int decode_tokens, float slo_us,
+                    float step_overhead_us, const int* chunks, int n_chunks, int* chunk_out,
+                    float* predicted_us);
 
 #ifdef __cplusplus
 }

@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 from tests.conftest import ROOT
@@ -124,4 +125,84 @@ def test_dispatch_table_default_set_save_load(S, tmp_path):
     bad.write_text("1 2 3\n")
     with pytest.raises(S.SpearError):
         S.dispatch_load(str(bad))
+    S.dispatch_clear()
+
+
+def test_dispatch_times_save_load_and_v1_lines(S, tmp_path):
+    S.dispatch_clear()
+    st = _layer(S, K=4096, N=4096, r=64)
+    with pytest.raises(S.SpearError):
+        S.dispatch_time_us(st, 8)                              # nothing measured yet
+    S.dispatch_set_time(4096, 4096, 64, 0, 8, S.PATH_DECODE, 12.5)
+    assert S.dispatch_time_us(st, 5) == pytest.approx(12.5)    # bucket 8
+    with pytest.raises(S.SpearError):
+        S.dispatch_set_time(4096, 4096, 64, 0, 8, S.PATH_DECODE, -1.0)
+    S.dispatch_set(4096, 4096, 64, 0, 64, S.PATH_FUSED)        # path only: no time
+    with pytest.raises(S.SpearError):
+        S.dispatch_time_us(st, 64)
+    p = tmp_path / "lut.txt"
+    S.dispatch_save(str(p))
+    S.dispatch_clear()
+    S.dispatch_load(str(p))
+    assert S.dispatch_time_us(st, 8) == pytest.approx(12.5)
+    assert S.F["spear_dispatch_choice"](ctypes.byref(st), 64) == S.PATH_FUSED
+    # a line without the time column loads as "not measured"
+    p.write_text(f"4096 4096 64 0 32 {S.PATH_UNFUSED}\n")
+    S.dispatch_clear()
+    S.dispatch_load(str(p))
+    assert S.F["spear_dispatch_choice"](ctypes.byref(st), 32) == S.PATH_UNFUSED
+    with pytest.raises(S.SpearError):
+        S.dispatch_time_us(st, 32)
+    S.dispatch_clear()
+
+
+def _brute_slo(times, decode, slo, overhead, chunks):
+    """Enumerate every candidate: predicted = overhead + sum of the layers'
+    tabled times at the power-of-two bucket of decode + chunk."""
+    fits = []
+    for c in chunks:
+        M = decode + c
+        if M < 1:
+            continue
+        b = 1
+        while b < M:
+            b *= 2
+        t = overhead + sum(tl[b] for tl in times)
+        if t <= slo:
+            fits.append((c, t))
+    if not fits:
+        return 0, -1.0
+    c = max(f[0] for f in fits)
+    return c, [f[1] for f in fits if f[0] == c][0]
+
+
+def test_slo_chunk_matches_enumeration(S):
+    S.dispatch_clear()
+    shapes = [(4096, 4096, 64, 0), (4096, 11008, 64, 0), (11008, 4096, 32, 128)]
+    buckets = [1 << i for i in range(13)]
+    rng = np.random.default_rng(7)
+    times = []
+    for (K, N, r, g) in shapes:
+        # monotone in M, like a measured latency table
+        t = np.cumsum(rng.uniform(0.5, 6.0, len(buckets))) + 5.0
+        times.append(dict(zip(buckets, t.tolist())))
+        for b, us in zip(buckets, t):
+            path = S.PATH_DECODE if b <= 16 else S.PATH_FUSED
+            S.dispatch_set_time(K, N, r, g, b, path, float(us))
+    layers = [_layer(S, K=K, N=N, r=r, group=g) for (K, N, r, g) in shapes]
+    chunks = [0, 16, 48, 64, 128, 256, 500, 1024, 2048]
+    for decode in (0, 1, 7, 16, 100):
+        for slo in (10.0, 40.0, 80.0, 150.0, 1e6):
+            got = S.slo_chunk(layers, decode, slo, chunks, step_overhead_us=3.0)
+            want = _brute_slo(times, decode, slo, 3.0, chunks)
+            assert got[0] == want[0], (decode, slo, got, want)
+            assert got[1] == pytest.approx(want[1], rel=1e-5)
+    # the loosest SLO takes the largest candidate, an impossible one takes none
+    assert S.slo_chunk(layers, 1, 1e6, chunks)[0] == 2048
+    assert S.slo_chunk(layers, 1, 1.0, chunks) == (0, -1.0)
+    # a bucket with no measured time is an error, not a guess
+    with pytest.raises(S.SpearError):
+        S.slo_chunk(layers, 1, 1e6, [8192])
+    with pytest.raises(S.SpearError):
+        S.slo_chunk(layers, 1, 100.0, [-4])
     S.dispatch_clear()

@@ -56,10 +56,16 @@ def test_dispatch_tune_picks_faster_path(S, shape, r, group):
         choice = S.dispatch_choice(layer, M)
         paths = [S.PATH_FUSED, S.PATH_UNFUSED] + ([S.PATH_DECODE] if M <= 16 else [])
         assert choice in paths
+        assert S.dispatch_time_us(layer, M) > 0.0     # tuning records the chosen path's time
         x = x_all[:M].contiguous()
         y = y_all[:M]
         t = {p: _median_us(S, layer, x, y, ws, p, flush) for p in paths}
         best = min(t.values())
         # within 5 % of the fastest, or within 2 us of it (timing noise at small M)
         assert t[choice] <= max(1.05 * best, best + 2.0), (M, choice, t)
+    # the SLO picker reads those times: with no overhead and an SLO equal to a
+    # bucket's time, that bucket's chunk is the largest that fits
+    t512 = S.dispatch_time_us(layer, 512)
+    chunk, pred = S.slo_chunk([layer], 0, t512, Ms)
+    assert pred <= t512 and chunk >= max(m for m in Ms if S.dispatch_time_us(layer, m) <= t512)
     S.dispatch_clear()

@@ -158,7 +158,11 @@ static WsLayout ws_layout(const LayerView& L, int M_max) {
 // ---------------------------------------------------------------------------
 using DKey = std::tuple<int, int, int, int, int>;  // K, N, r, group, M bucket
 static std::mutex g_dmu;
-static std::map<DKey, int> g_table;
+struct DEntry {
+  int path;
+  float us;  // measured time of that path at the bucket's M, < 0 if not measured
+};
+static std::map<DKey, DEntry> g_table;
 
 static int m_bucket(int M) {
   int b = 1;
@@ -176,7 +180,7 @@ static int choose_path(const LayerView& L, int M) {
     std::lock_guard<std::mutex> lk(g_dmu);
     auto it = g_table.find(DKey(L.K, L.N, L.r, L.group, m_bucket(M)));
     if (it != g_table.end()) {
-      const int p = it->second;
+      const int p = it->second.path;
       if (!(p == SPEAR_PATH_DECODE && M > 16)) return p;
     }
   }
@@ -418,7 +422,77 @@ int spear_dispatch_set(int K, int N, int r, int group, int M, int path) {
   if (M < 1) return set_error(SPEAR_ERR_INVALID_ARG, "bad M");
   if (path == SPEAR_PATH_DECODE && M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs M <= 16");
   std::lock_guard<std::mutex> lk(g_dmu);
-  g_table[DKey(K, N, r, group, m_bucket(M))] = path;
+  g_table[DKey(K, N, r, group, m_bucket(M))] = DEntry{path, -1.f};
+  return SPEAR_OK;
+}
+
+int spear_dispatch_set_time(int K, int N, int r, int group, int M, int path, float us) {
+  g_last_error.clear();
+  if (!(us >= 0.f)) return set_error(SPEAR_ERR_INVALID_ARG, "time must be >= 0 us");
+  const int rc = spear_dispatch_set(K, N, r, group, M, path);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lk(g_dmu);
+  g_table[DKey(K, N, r, group, m_bucket(M))].us = us;
+  return SPEAR_OK;
+}
+
+int spear_dispatch_time_us(const spear_layer* layer, int M, float* us) {
+  g_last_error.clear();
+  LayerView L;
+  int rc = check_layer(layer, &L);
+  if (rc) return rc;
+  if (M < 1 || !us) return set_error(SPEAR_ERR_INVALID_ARG, "bad M or NULL output");
+  std::lock_guard<std::mutex> lk(g_dmu);
+  auto it = g_table.find(DKey(L.K, L.N, L.r, L.group, m_bucket(M)));
+  if (it == g_table.end() || it->second.us < 0.f)
+    return set_error(SPEAR_ERR_INVALID_ARG, "no measured time for K=%d N=%d r=%d group=%d at M bucket %d", L.K, L.N,
+                     L.r, L.group, m_bucket(M));
+  *us = it->second.us;
+  return SPEAR_OK;
+}
+
+// SLO-constrained chunk size (SPEAR, gist.science technical summary, section
+// 2.2 C: the scheduler picks the largest prefill chunk that meets the
+// inter-token latency SLO, from precomputed kernel latency tables).  A step
+// runs decode_tokens + chunk tokens through every layer; its predicted time is
+// step_overhead_us plus the table time of each layer at the step's M bucket
+// (the bucket rounds M up, so the prediction is the bucket's measured time).
+int spear_slo_chunk(const spear_layer* const* layers, int n_layers, int decode_tokens, float slo_us,
+                    float step_overhead_us, const int* chunks, int n_chunks, int* chunk_out, float* predicted_us) {
+  g_last_error.clear();
+  if (!layers || n_layers <= 0 || !chunks || n_chunks <= 0 || !chunk_out)
+    return set_error(SPEAR_ERR_INVALID_ARG, "NULL or empty argument");
+  if (decode_tokens < 0 || !(slo_us > 0.f) || !(step_overhead_us >= 0.f))
+    return set_error(SPEAR_ERR_INVALID_ARG, "bad decode_tokens, SLO or overhead");
+  std::vector<LayerView> Ls(n_layers);
+  for (int l = 0; l < n_layers; ++l) {
+    int rc = check_layer(layers[l], &Ls[l]);
+    if (rc) return rc;
+  }
+  int best = 0;
+  float best_t = -1.f;
+  std::lock_guard<std::mutex> lk(g_dmu);
+  for (int c = 0; c < n_chunks; ++c) {
+    const int chunk = chunks[c];
+    if (chunk < 0) return set_error(SPEAR_ERR_INVALID_ARG, "negative chunk size");
+    const int M = decode_tokens + chunk;
+    if (M < 1) continue;
+    float t = step_overhead_us;
+    for (int l = 0; l < n_layers; ++l) {
+      const LayerView& L = Ls[l];
+      auto it = g_table.find(DKey(L.K, L.N, L.r, L.group, m_bucket(M)));
+      if (it == g_table.end() || it->second.us < 0.f)
+        return set_error(SPEAR_ERR_INVALID_ARG, "layer %d (K=%d N=%d r=%d group=%d) has no measured time at M bucket %d",
+                         l, L.K, L.N, L.r, L.group, m_bucket(M));
+      t += it->second.us;
+    }
+    if (t <= slo_us && chunk >= best) {
+      if (chunk > best || best_t < 0.f) best_t = t;
+      best = chunk;
+    }
+  }
+  *chunk_out = best;
+  if (predicted_us) *predicted_us = best_t;
   return SPEAR_OK;
 }
 
@@ -433,10 +507,10 @@ int spear_dispatch_save(const char* path) {
   FILE* f = fopen(path, "w");
   if (!f) return set_error(SPEAR_ERR_INVALID_ARG, "cannot open %s for writing", path);
   std::lock_guard<std::mutex> lk(g_dmu);
-  fprintf(f, "# spear dispatch table v1: K N r group M_bucket path\n");
+  fprintf(f, "# spear dispatch table v2: K N r group M_bucket path time_us (-1 = not measured)\n");
   for (const auto& kv : g_table)
-    fprintf(f, "%d %d %d %d %d %d\n", std::get<0>(kv.first), std::get<1>(kv.first), std::get<2>(kv.first),
-            std::get<3>(kv.first), std::get<4>(kv.first), kv.second);
+    fprintf(f, "%d %d %d %d %d %d %.3f\n", std::get<0>(kv.first), std::get<1>(kv.first), std::get<2>(kv.first),
+            std::get<3>(kv.first), std::get<4>(kv.first), kv.second.path, kv.second.us);
   fclose(f);
   return SPEAR_OK;
 }
@@ -446,19 +520,20 @@ int spear_dispatch_load(const char* path) {
   if (!path) return set_error(SPEAR_ERR_INVALID_ARG, "NULL path");
   FILE* f = fopen(path, "r");
   if (!f) return set_error(SPEAR_ERR_INVALID_ARG, "cannot open %s", path);
-  std::map<DKey, int> t;
+  std::map<DKey, DEntry> t;
   char line[256];
   int lineno = 0;
   while (fgets(line, sizeof(line), f)) {
     ++lineno;
     if (line[0] == '#' || line[0] == '\n') continue;
     int K, N, r, g, mb, p;
-    if (sscanf(line, "%d %d %d %d %d %d", &K, &N, &r, &g, &mb, &p) != 6 || p < SPEAR_PATH_DECODE ||
-        p > SPEAR_PATH_UNFUSED || mb < 1) {
+    float us = -1.f;
+    const int n = sscanf(line, "%d %d %d %d %d %d %f", &K, &N, &r, &g, &mb, &p, &us);
+    if ((n != 6 && n != 7) || p < SPEAR_PATH_DECODE || p > SPEAR_PATH_UNFUSED || mb < 1) {
       fclose(f);
       return set_error(SPEAR_ERR_INVALID_ARG, "%s:%d: malformed entry", path, lineno);
     }
-    t[DKey(K, N, r, g, mb)] = p;
+    t[DKey(K, N, r, g, mb)] = DEntry{p, us};
   }
   fclose(f);
   std::lock_guard<std::mutex> lk(g_dmu);
@@ -530,7 +605,7 @@ int spear_dispatch_tune(const spear_layer* layer, const int* Ms, int nM, const u
     }
     if (result == SPEAR_OK) {
       std::lock_guard<std::mutex> lk(g_dmu);
-      g_table[DKey(L.K, L.N, L.r, L.group, m_bucket(M))] = best_path;
+      g_table[DKey(L.K, L.N, L.r, L.group, m_bucket(M))] = DEntry{best_path, best < 1e29f ? best : -1.f};
     }
   }
   cudaEventDestroy(e0);

@@ -79,9 +79,13 @@ EXPORTS = {
     "spear_dispatch_tune": (_i, ctypes.POINTER(LayerStruct), ctypes.POINTER(_i), _i, _vp, _vp, _vp, _sz, _vp, _sz,
                             _i, ctypes.POINTER(_f), _vp),
     "spear_dispatch_set": (_i, _i, _i, _i, _i, _i, _i),
+    "spear_dispatch_set_time": (_i, _i, _i, _i, _i, _i, _i, _f),
+    "spear_dispatch_time_us": (_i, ctypes.POINTER(LayerStruct), _i, ctypes.POINTER(_f)),
     "spear_dispatch_clear": (None,),
     "spear_dispatch_save": (_i, ctypes.c_char_p),
     "spear_dispatch_load": (_i, ctypes.c_char_p),
+    "spear_slo_chunk": (_i, ctypes.POINTER(ctypes.POINTER(LayerStruct)), _i, _i, _f, _f, ctypes.POINTER(_i), _i,
+                        ctypes.POINTER(_i), ctypes.POINTER(_f)),
 }
 
 F = {name: _proto(name, sig[0], *sig[1:]) for name, sig in EXPORTS.items()}
@@ -287,6 +291,31 @@ def dispatch_tune(layer: Layer, Ms: list[int], x: torch.Tensor, y: torch.Tensor,
 
 def dispatch_set(K: int, N: int, r: int, group: int, M: int, path: int) -> None:
     _check(F["spear_dispatch_set"](K, N, r, group, M, path))
+
+
+def dispatch_set_time(K: int, N: int, r: int, group: int, M: int, path: int, us: float) -> None:
+    _check(F["spear_dispatch_set_time"](K, N, r, group, M, path, us))
+
+
+def dispatch_time_us(layer, M: int) -> float:
+    st = layer.struct() if hasattr(layer, "struct") else layer
+    out = _f()
+    _check(F["spear_dispatch_time_us"](ctypes.byref(st), M, ctypes.byref(out)))
+    return float(out.value)
+
+
+def slo_chunk(layers: list, decode_tokens: int, slo_us: float, chunks: list[int],
+              step_overhead_us: float = 0.0) -> tuple[int, float]:
+    """Largest candidate prefill chunk whose predicted step time (overhead plus
+    every layer's tabled time at M = decode_tokens + chunk) meets ``slo_us``;
+    returns (chunk, predicted_us), (0, -1) if none fits."""
+    structs = [l.struct() if hasattr(l, "struct") else l for l in layers]
+    ptrs = (ctypes.POINTER(LayerStruct) * len(structs))(*[ctypes.pointer(s) for s in structs])
+    arr = (_i * len(chunks))(*chunks)
+    out, pred = _i(), _f()
+    _check(F["spear_slo_chunk"](ptrs, len(structs), decode_tokens, slo_us, step_overhead_us, arr, len(chunks),
+                                ctypes.byref(out), ctypes.byref(pred)))
+    return int(out.value), float(pred.value)
 
 
 def dispatch_clear() -> None:
