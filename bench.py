@@ -500,7 +500,7 @@ def run_sweep(args):
                 ts.append(a.elapsed_time(b) * 1e3)
         return float(np.median(ts))
 
-    names = {S.PATH_DECODE: "decode", S.PATH_FUSED: "fused", S.PATH_UNFUSED: "unfused"}
+    names = S.PATH_NAMES
     points, good = [], 0
     S.dispatch_clear()
     t_start = time.perf_counter()
@@ -516,7 +516,7 @@ def run_sweep(args):
                 y_all = torch.empty((max(SWEEP_MS), N), dtype=torch.bfloat16, device="cuda")
                 S.dispatch_tune(layer, list(SWEEP_MS), x_all, y_all, ws, flush=flush, reps=10)
                 for M in SWEEP_MS:
-                    paths = [S.PATH_FUSED, S.PATH_UNFUSED] + ([S.PATH_DECODE] if M <= 16 else [])
+                    paths = [S.PATH_FUSED, S.PATH_UNFUSED, S.PATH_SEMIFUSED] + ([S.PATH_DECODE] if M <= 16 else [])
                     x = x_all[:M].contiguous()
                     t = {p: median_us(layer, x, y_all[:M], ws, p, 10) for p in paths}
                     choice = S.dispatch_choice(layer, M)

@@ -61,7 +61,16 @@ enum {
   SPEAR_PATH_AUTO = 0,    /* dispatcher's choice                                   */
   SPEAR_PATH_DECODE = 1,  /* split-K GEMV kernel with the EC fused (M <= 16)       */
   SPEAR_PATH_FUSED = 2,   /* tcgen05 GEMM with the EC fused into the same kernel   */
-  SPEAR_PATH_UNFUSED = 3  /* GEMM with the EC disabled, then a separate EC kernel  */
+  SPEAR_PATH_UNFUSED = 3, /* GEMM with the EC disabled, then a separate EC kernel  */
+  SPEAR_PATH_SEMIFUSED = 4 /* SPEAR's prefill DAG (gist.science technical summary,
+                            * section 2.2 A): the EC projection (g, g*t) on a
+                            * second, high-priority stream concurrently with the
+                            * EC-disabled GEMM on `stream`, then the in-place
+                            * update g*(t.B) after both.  The fork and join are
+                            * CUDA events, so capturing `stream` into a CUDA
+                            * graph captures the two-branch DAG.  One side stream
+                            * per device, shared by all callers: host enqueue of
+                            * this path is serialised by a mutex. */
 };
 
 /* Message of the last failing call on this host thread ("" if none). */
@@ -216,8 +225,9 @@ int spear_dispatch_choice(const spear_layer* layer, int M);
  * (median of `reps` runs, each preceded by writing flush_bytes of the
  * optional device buffer `flush` to evict L2) and record the fastest in the
  * table.  x: device bf16 M_max x K input, y: device bf16 M_max x N scratch
- * output (M_max = max of Ms).  times_us (optional host array [nM*3]) receives
- * the median of each path (DECODE, FUSED, UNFUSED; negative = not run).
+ * output (M_max = max of Ms).  times_us (optional host array [nM*4]) receives
+ * the median of each path (DECODE, FUSED, UNFUSED, SEMIFUSED; negative = not
+ * run).
  * Synchronises the stream. */
 int spear_dispatch_tune(const spear_layer* layer, const int* Ms, int nM,
                         const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes,

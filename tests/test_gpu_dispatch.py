@@ -54,7 +54,7 @@ def test_dispatch_tune_picks_faster_path(S, shape, r, group):
     assert S.read_status(ws) == S.OK
     for M in Ms:
         choice = S.dispatch_choice(layer, M)
-        paths = [S.PATH_FUSED, S.PATH_UNFUSED] + ([S.PATH_DECODE] if M <= 16 else [])
+        paths = [S.PATH_FUSED, S.PATH_UNFUSED, S.PATH_SEMIFUSED] + ([S.PATH_DECODE] if M <= 16 else [])
         assert choice in paths
         assert S.dispatch_time_us(layer, M) > 0.0     # tuning records the chosen path's time
         x = x_all[:M].contiguous()

@@ -188,6 +188,38 @@ static int choose_path(const LayerView& L, int M) {
 }
 
 // ---------------------------------------------------------------------------
+// semi-fused prefill: a side stream per device and the fork / join events
+// ---------------------------------------------------------------------------
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+static std::mutex g_side_mu;  // held from the fork to the join of one call
+
+static int side_stream(SideStream** out) {
+  static std::map<int, SideStream> streams;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return set_cuda_error("get device", e);
+  SideStream& ss = streams[dev];
+  if (!ss.s) {
+    int lo = 0, hi = 0;
+    cudaDeviceGetStreamPriorityRange(&lo, &hi);
+    // the projection is short and lies on the DAG's critical path: its CTAs
+    // go to the block scheduler ahead of the GEMM's tiles
+    e = cudaStreamCreateWithPriority(&ss.s, cudaStreamNonBlocking, hi);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      ss = SideStream{};
+      return set_cuda_error("side stream create", e);
+    }
+  }
+  *out = &ss;
+  return SPEAR_OK;
+}
+
+// ---------------------------------------------------------------------------
 // forward
 // ---------------------------------------------------------------------------
 static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, uint8_t* ws,
@@ -242,6 +274,36 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
     EcPlan ep = plan_ec(M, L.K, L.N, L.r, sms);
     return launch_ec(ep, L, x, M, y, hdr, part, tickets, mflags, gt, gate_out, mask_count, st);
   }
+  if (path == SPEAR_PATH_SEMIFUSED) {
+    LayerView L0 = L;
+    L0.r = 0;
+    L0.agt = nullptr;
+    L0.bpt = nullptr;
+    const bool d2 = M <= 16 && !decode2_unsupported(M, L.K, L.N, L.r);
+    auto gemm = [&](float* go, int* mc) {
+      if (d2) return launch_decode2(L0, x, M, y, hdr, tbuf, go, mc, false, st);
+      TcPlan p = plan_tc(M, L.K, L.N, 0, L.group, sms);
+      return launch_tc(p, L0, x, M, y, false, hdr, tcflags, gt, go, mc, st);
+    };
+    if (L.r == 0) return gemm(gate_out, mask_count);
+    const EcPlan ep = plan_ec(M, L.K, L.N, L.r, sms);
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    SideStream* ss = nullptr;
+    int rc = side_stream(&ss);
+    if (rc) return rc;
+    cudaError_t e = cudaEventRecord(ss->fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->s, ss->fork, 0);
+    if (e != cudaSuccess) return set_cuda_error("semi-fused fork", e);
+    rc = launch_ec(ep, L, x, M, y, hdr, part, tickets, mflags, gt, gate_out, mask_count, ss->s, 1);
+    e = cudaEventRecord(ss->join, ss->s);
+    // the GEMM goes on `st` after the fork only, so it runs beside the projection
+    if (rc == SPEAR_OK && e == cudaSuccess) rc = gemm(nullptr, nullptr);
+    // join on every return, so a capture of `st` never loses the side branch
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ss->join, 0);
+    if (e != cudaSuccess) return set_cuda_error("semi-fused join", e);
+    if (rc) return rc;
+    return launch_ec(ep, L, x, M, y, hdr, part, tickets, mflags, gt, nullptr, nullptr, st, 2);
+  }
   if (path == SPEAR_PATH_FUSED) {
     TcPlan p = plan_tc(M, L.K, L.N, L.r, L.group, sms);
     return launch_tc(p, L, x, M, y, L.r > 0, hdr, tcflags, gt, gate_out, mask_count, st);
@@ -259,7 +321,8 @@ static int forward_impl(const spear_layer* layer, const uint16_t* x, int M, uint
   if (!aligned16(x) || !aligned16(y) || !aligned16(ws) || (gate_out && ((uintptr_t)gate_out & 3)) ||
       (mask_count && ((uintptr_t)mask_count & 3)))
     return set_error(SPEAR_ERR_ALIGNMENT, "x, y, ws must be 16-byte aligned");
-  if (path < SPEAR_PATH_AUTO || path > SPEAR_PATH_UNFUSED) return set_error(SPEAR_ERR_INVALID_ARG, "bad path %d", path);
+  if (path < SPEAR_PATH_AUTO || path > SPEAR_PATH_SEMIFUSED)
+    return set_error(SPEAR_ERR_INVALID_ARG, "bad path %d", path);
   const WsLayout wl = ws_layout(L, M);
   if (ws_bytes < wl.total)
     return set_error(SPEAR_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed for M=%d", ws_bytes, wl.total, M);
@@ -418,7 +481,7 @@ int spear_dispatch_choice(const spear_layer* layer, int M) {
 
 int spear_dispatch_set(int K, int N, int r, int group, int M, int path) {
   g_last_error.clear();
-  if (path < SPEAR_PATH_DECODE || path > SPEAR_PATH_UNFUSED) return set_error(SPEAR_ERR_INVALID_ARG, "bad path");
+  if (path < SPEAR_PATH_DECODE || path > SPEAR_PATH_SEMIFUSED) return set_error(SPEAR_ERR_INVALID_ARG, "bad path");
   if (M < 1) return set_error(SPEAR_ERR_INVALID_ARG, "bad M");
   if (path == SPEAR_PATH_DECODE && M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs M <= 16");
   std::lock_guard<std::mutex> lk(g_dmu);
@@ -529,7 +592,7 @@ int spear_dispatch_load(const char* path) {
     int K, N, r, g, mb, p;
     float us = -1.f;
     const int n = sscanf(line, "%d %d %d %d %d %d %f", &K, &N, &r, &g, &mb, &p, &us);
-    if ((n != 6 && n != 7) || p < SPEAR_PATH_DECODE || p > SPEAR_PATH_UNFUSED || mb < 1) {
+    if ((n != 6 && n != 7) || p < SPEAR_PATH_DECODE || p > SPEAR_PATH_SEMIFUSED || mb < 1) {
       fclose(f);
       return set_error(SPEAR_ERR_INVALID_ARG, "%s:%d: malformed entry", path, lineno);
     }
@@ -565,8 +628,8 @@ int spear_dispatch_tune(const spear_layer* layer, const int* Ms, int nM, const u
     const int M = Ms[i];
     float best = 1e30f;
     int best_path = default_path(L, M);
-    const int paths[3] = {SPEAR_PATH_DECODE, SPEAR_PATH_FUSED, SPEAR_PATH_UNFUSED};
-    for (int pi = 0; pi < 3; ++pi) {
+    const int paths[4] = {SPEAR_PATH_DECODE, SPEAR_PATH_FUSED, SPEAR_PATH_UNFUSED, SPEAR_PATH_SEMIFUSED};
+    for (int pi = 0; pi < 4; ++pi) {
       const int path = paths[pi];
       float med = -1.f;
       if (!(path == SPEAR_PATH_DECODE && M > 16)) {
@@ -601,7 +664,7 @@ int spear_dispatch_tune(const spear_layer* layer, const int* Ms, int nM, const u
           g_last_error.clear();
         }
       }
-      if (times_us) times_us[i * 3 + pi] = med;
+      if (times_us) times_us[i * 4 + pi] = med;
     }
     if (result == SPEAR_OK) {
       std::lock_guard<std::mutex> lk(g_dmu);

@@ -25,7 +25,9 @@ struct WsHeader {
   int ec_flag;    // == epoch + 1 once the gated EC projection of this launch is ready
   int d2_epoch;   // decode path: launches completed (tags its EC projection words)
   int gt_obs;     // decode path: CTAs that have read the complete EC projection
-  int pad0[57];
+  int sf_done;    // semi-fused EC projection launch: CTAs finished
+  int sf_count;   // semi-fused EC projection launch: tokens with g < tau
+  int pad0[55];
 };
 static_assert(sizeof(WsHeader) <= 256, "header must fit in 256 bytes");
 constexpr size_t kWsHeaderBytes = 256;

@@ -15,6 +15,12 @@
 //    and read-modify-writes y.
 // Items are processed in increasing order by every warp, so A items never
 // wait and B items only wait on A items that are already being processed.
+//
+// The same kernel also runs as two launches (phase 1: A items only, phase 2:
+// B items only), which is the semi-fused prefill DAG: phase 1 on a second
+// stream concurrently with the EC-disabled GEMM, phase 2 after both.  Stream
+// order then replaces the m-block flags, so neither phase waits on the device
+// and neither needs its CTAs co-resident.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -40,6 +46,7 @@ struct EcArgs {
   float b_g, tau;
   int ksplit, RT, Mb16, Mpad, E;
   int itemsA, itemsB;
+  int phase;         // 0: both item kinds in one launch, 1: A items only, 2: B items only
 };
 
 __device__ __forceinline__ uint32_t w8(const uint4& a, const uint4& b, int i) {
@@ -157,9 +164,11 @@ __device__ void ec_item_project(const EcArgs& a, int item, int lane, int epoch) 
   __syncwarp();
   if (lane == 0) {
     a.tickets[mb] = 0;
-    if (a.mask_count) atomicAdd(&a.hdr->ec_done, __popc(below));
-    __threadfence();
-    st_release_gpu(&a.mflags[mb], epoch + 1);
+    if (a.mask_count) atomicAdd(a.phase == 0 ? &a.hdr->ec_done : &a.hdr->sf_count, __popc(below));
+    if (a.phase == 0) {
+      __threadfence();
+      st_release_gpu(&a.mflags[mb], epoch + 1);
+    }
   }
 }
 
@@ -210,7 +219,7 @@ __device__ void ec_item_update(const EcArgs& a, int item, int lane, int epoch, _
   const int m0 = mb64 * 64;
   const int rho = lane >> 2, cq = lane & 3;
   bool ok = true;
-  if (lane < 4) {
+  if (a.phase == 0 && lane < 4) {
     const int mb = mb64 * 4 + lane;
     if (mb < a.Mb16) ok = wait_flag_eq(&a.mflags[mb], epoch + 1, a.hdr);
   }
@@ -280,7 +289,21 @@ __global__ void __launch_bounds__(EC_WARPS * 32) ec_kernel(const __grid_constant
     else
       ec_item_update(a, it - a.itemsA, lane, epoch, stage_all[warp]);
   }
+  if (a.phase == 2) return;
   __syncthreads();
+  if (a.phase == 1) {
+    if (threadIdx.x == 0 && a.mask_count) {
+      __threadfence();
+      const int prev = atomicAdd(&a.hdr->sf_done, 1);
+      if (prev == (int)gridDim.x - 1) {
+        __threadfence();
+        *a.mask_count = *reinterpret_cast<volatile int*>(&a.hdr->sf_count);
+        a.hdr->sf_done = 0;
+        a.hdr->sf_count = 0;
+      }
+    }
+    return;
+  }
   if (threadIdx.x == 0) {
     __threadfence();
     const int prev = atomicAdd(&a.hdr->done_ctas, 1);
@@ -313,7 +336,7 @@ EcPlan plan_ec(int M, int K, int N, int r, int sm_count) {
 
 int launch_ec(const EcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, WsHeader* hdr,
               float* part, int* tickets, int* mflags, __nv_bfloat16* gt, float* gate_out, int* mask_count,
-              cudaStream_t st) {
+              cudaStream_t st, int phase) {
   EcArgs a = {};
   a.x = x;
   a.y = y;
@@ -339,8 +362,9 @@ int launch_ec(const EcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
   a.Mb16 = (M + 15) / 16;
   a.Mpad = ((M + 63) / 64) * 64;
   a.E = (L.r + 16) / 16;
-  a.itemsA = a.Mb16 * p.ksplit;
-  a.itemsB = (a.Mpad / 64) * (L.N / 32);
+  a.itemsA = phase == 2 ? 0 : a.Mb16 * p.ksplit;
+  a.itemsB = phase == 1 ? 0 : (a.Mpad / 64) * (L.N / 32);
+  a.phase = phase;
   // every CTA must be resident at once: B items wait for A items of other CTAs
   static int per_sm = 0;
   if (per_sm == 0) {
@@ -351,7 +375,13 @@ int launch_ec(const EcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = p.grid < per_sm * sms ? p.grid : per_sm * sms;
+  int grid = p.grid < per_sm * sms ? p.grid : per_sm * sms;
+  if (phase != 0) {
+    // split phases never wait on one another's CTAs: no residency cap, and
+    // no more CTAs than the items need
+    const int need = (a.itemsA + a.itemsB + EC_WARPS - 1) / EC_WARPS;
+    grid = need < p.grid ? need : p.grid;
+  }
   ec_kernel<<<grid, EC_WARPS * 32, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPEAR_OK : set_cuda_error("ec kernel launch", e);

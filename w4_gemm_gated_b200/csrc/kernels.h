@@ -59,6 +59,8 @@ int launch_decode2(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloa
                    float* gate_out, int* mask_count, bool ec_only, cudaStream_t st);
 
 // ---- standalone EC kernel (ec.cu): y += g * (x.A).B, in place ----
+// phase 0: one launch; 1: projection (gt, gate, mask count) only; 2: the
+// in-place update only, after a phase-1 launch that stream order completed
 struct EcPlan {
   int ksplit;   // K parts of the projection
   int grid;     // persistent CTAs
@@ -68,7 +70,7 @@ struct EcPlan {
 EcPlan plan_ec(int M, int K, int N, int r, int sm_count);
 int launch_ec(const EcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y,
               WsHeader* hdr, float* part, int* tickets, int* mflags, __nv_bfloat16* gt, float* gate_out,
-              int* mask_count, cudaStream_t st);
+              int* mask_count, cudaStream_t st, int phase = 0);
 
 // ---- tensor-core path (tc_gemm.cu) ----
 struct TcPlan {

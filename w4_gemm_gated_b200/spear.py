@@ -31,7 +31,8 @@ PATH_AUTO = 0
 PATH_DECODE = 1
 PATH_FUSED = 2
 PATH_UNFUSED = 3
-PATH_NAMES = {PATH_DECODE: "decode", PATH_FUSED: "fused", PATH_UNFUSED: "unfused"}
+PATH_SEMIFUSED = 4
+PATH_NAMES = {PATH_DECODE: "decode", PATH_FUSED: "fused", PATH_UNFUSED: "unfused", PATH_SEMIFUSED: "semifused"}
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -279,14 +280,15 @@ def dispatch_choice(layer: Layer, M: int) -> int:
 
 
 def dispatch_tune(layer: Layer, Ms: list[int], x: torch.Tensor, y: torch.Tensor, ws: torch.Tensor,
-                  flush: torch.Tensor | None = None, reps: int = 20, stream=None) -> list[tuple[float, float, float]]:
+                  flush: torch.Tensor | None = None, reps: int = 20, stream=None) -> list[tuple[float, ...]]:
+    """Median microseconds per M of (DECODE, FUSED, UNFUSED, SEMIFUSED), -1 where not run."""
     st = layer.struct()
     arr = (_i * len(Ms))(*Ms)
-    times = (_f * (3 * len(Ms)))()
+    times = (_f * (4 * len(Ms)))()
     _check(F["spear_dispatch_tune"](ctypes.byref(st), arr, len(Ms), _ptr(x), _ptr(y), _ptr(ws), ws.numel(),
                                     _ptr(flush), 0 if flush is None else flush.numel() * flush.element_size(),
                                     reps, times, _stream(stream)))
-    return [(times[3 * i], times[3 * i + 1], times[3 * i + 2]) for i in range(len(Ms))]
+    return [tuple(times[4 * i + j] for j in range(4)) for i in range(len(Ms))]
 
 
 def dispatch_set(K: int, N: int, r: int, group: int, M: int, path: int) -> None:
