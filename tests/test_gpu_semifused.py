@@ -1,8 +1,9 @@
 """GPU parity of the semi-fused prefill path: the EC projection on a second
 stream beside the EC-disabled GEMM, then the in-place EC update (SPEAR,
 gist.science technical summary, section 2.2 A).  Checked against the CPU
-oracle, bit for bit against the one-launch unfused EC (same arithmetic, other
-schedule), and under CUDA-graph capture of the two-branch DAG."""
+oracle, bit for bit against the unfused path (the same EC launches after the
+GEMM instead of beside it), and under CUDA-graph capture of the two-branch
+DAG."""
 import numpy as np
 import pytest
 import torch

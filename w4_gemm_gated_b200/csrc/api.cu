@@ -93,7 +93,7 @@ int device_sm_count() { return sm_count(); }
 // workspace layout
 // ---------------------------------------------------------------------------
 struct WsLayout {
-  size_t hdr, mflags, tickets, tcflags, t, gt, part, total;
+  size_t hdr, tickets, tcflags, t, gt, part, total;
   int n_flags;
 };
 
@@ -113,8 +113,6 @@ static WsLayout ws_layout_uncached(const LayerView& L, int M_max) {
   w.n_flags = kFlagCap;
   size_t off = kWsHeaderBytes;
   w.hdr = 0;
-  w.mflags = off;
-  off = up256(off + sizeof(int) * kFlagCap);
   w.tickets = off;
   off = up256(off + sizeof(int) * kFlagCap);
   w.tcflags = off;
@@ -225,7 +223,6 @@ static int side_stream(SideStream** out) {
 static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, uint8_t* ws,
                     const WsLayout& wl, float* gate_out, int* mask_count, int path, cudaStream_t st) {
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + wl.hdr);
-  int* mflags = reinterpret_cast<int*>(ws + wl.mflags);
   int* tickets = reinterpret_cast<int*>(ws + wl.tickets);
   int* tcflags = reinterpret_cast<int*>(ws + wl.tcflags);
   float* tbuf = reinterpret_cast<float*>(ws + wl.t);
@@ -271,8 +268,11 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
                      L.r > 0 ? nullptr : mask_count, st);
     }
     if (rc || L.r == 0) return rc;
+    // the separate EC kernel: projection and gate, then the update of y
     EcPlan ep = plan_ec(M, L.K, L.N, L.r, sms);
-    return launch_ec(ep, L, x, M, y, hdr, part, tickets, mflags, gt, gate_out, mask_count, st);
+    rc = launch_ec(ep, L, x, M, y, hdr, part, tickets, gt, gate_out, mask_count, st, 1);
+    if (rc) return rc;
+    return launch_ec(ep, L, x, M, y, hdr, part, tickets, gt, nullptr, nullptr, st, 2);
   }
   if (path == SPEAR_PATH_SEMIFUSED) {
     LayerView L0 = L;
@@ -294,7 +294,7 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
     cudaError_t e = cudaEventRecord(ss->fork, st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->s, ss->fork, 0);
     if (e != cudaSuccess) return set_cuda_error("semi-fused fork", e);
-    rc = launch_ec(ep, L, x, M, y, hdr, part, tickets, mflags, gt, gate_out, mask_count, ss->s, 1);
+    rc = launch_ec(ep, L, x, M, y, hdr, part, tickets, gt, gate_out, mask_count, ss->s, 1);
     e = cudaEventRecord(ss->join, ss->s);
     // the GEMM goes on `st` after the fork only, so it runs beside the projection
     if (rc == SPEAR_OK && e == cudaSuccess) rc = gemm(nullptr, nullptr);
@@ -302,7 +302,7 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
     if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ss->join, 0);
     if (e != cudaSuccess) return set_cuda_error("semi-fused join", e);
     if (rc) return rc;
-    return launch_ec(ep, L, x, M, y, hdr, part, tickets, mflags, gt, nullptr, nullptr, st, 2);
+    return launch_ec(ep, L, x, M, y, hdr, part, tickets, gt, nullptr, nullptr, st, 2);
   }
   if (path == SPEAR_PATH_FUSED) {
     TcPlan p = plan_tc(M, L.K, L.N, L.r, L.group, sms);

@@ -5,10 +5,10 @@
 // memory-bound decode phase (gist.science technical summary, section 2.2 A,
 // decode at M = 1: one kernel, no inter-kernel launch on the critical path).
 //
-// Residency.  One CTA per SM per launch, sized to half an SM (192 threads, at
-// most 112 KB of shared memory), so that the next launch in the stream
-// (programmatic dependent launch) sits beside it on the same SM and streams
-// its own weights while this one finishes.
+// Residency.  Two CTAs per SM per launch, each half an SM (192 threads, at
+// most 112 KB of shared memory), so the whole grid is resident at once.  The
+// next launch in the stream (programmatic dependent launch) takes an SM's
+// halves as this one leaves them and streams its own weights before it waits.
 //
 // Split.  K is cut into CS parts, one per CTA of a cluster, and each part into
 // 4 warp slices of KTW 64-wide k-tiles.  A consumer warp loads the activations
@@ -990,8 +990,9 @@ static D2Plan make_d2_plan(int MT, int K, int N, int r, int sms) {
   p.KTP = KT / p.CS;
   p.ES = r > 0 ? (r + 1 + 15) / 16 : 0;
   const int NS = N / 16;
-  // one CTA per SM per launch
-  int NC = std::max(1, sms / p.CS);
+  // two CTAs per SM per launch: the next launch takes an SM's halves as this
+  // one leaves them (measured faster than one CTA per SM beside the next launch)
+  int NC = std::max(1, 2 * sms / p.CS);
   NC = std::min(NC, std::max(1, NS + p.ES));
   NC = std::min(NC, D2_MAXCL);
   p.NC = NC;

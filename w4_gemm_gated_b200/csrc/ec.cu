@@ -1,26 +1,21 @@
-// Standalone Error-Compensator kernel of the unfused path:
+// Standalone Error-Compensator kernel of the unfused and semi-fused paths:
 //     y <- bf16( y + g * ((x . A) . B) )     (in place)
 // SPEAR runs the EC of the compute-bound prefill phase as a kernel of its own
 // next to the low-bit GEMM (gist.science technical summary, section 2.2 A,
-// "chemin semi-fusionne"); this is that kernel, run after a GEMM whose own EC
-// is disabled.
+// "chemin semi-fusionne"); this is that kernel, run beside or after a GEMM
+// whose own EC is disabled.
 //
-// One persistent launch, two kinds of warp work items, projection items first:
-//  A (m-block of 16 tokens, K part): partial [t | logit] = x . [A | w_g] on the
-//    tensor cores (mma.sync), written to a partial buffer; the last of the K
-//    parts (ticket) sums the parts in a fixed order, applies the gate and
-//    publishes gt = g * t (bf16) with an epoch-tagged flag for the m-block.
-//  B (64 tokens, 32 output channels): waits (bounded) for its four m-block
-//    flags, computes gt . B' with MMA k-steps, scales by s_n (per-channel fold)
-//    and read-modify-writes y.
-// Items are processed in increasing order by every warp, so A items never
-// wait and B items only wait on A items that are already being processed.
-//
-// The same kernel also runs as two launches (phase 1: A items only, phase 2:
-// B items only), which is the semi-fused prefill DAG: phase 1 on a second
-// stream concurrently with the EC-disabled GEMM, phase 2 after both.  Stream
-// order then replaces the m-block flags, so neither phase waits on the device
-// and neither needs its CTAs co-resident.
+// Two launches, one kind of warp work item each:
+//  phase 1, A items (m-block of 16 tokens, K part): partial [t | logit] =
+//    x . [A | w_g] on the tensor cores (mma.sync), written to a partial
+//    buffer; the last of the K parts (ticket) sums the parts in a fixed order,
+//    applies the gate and writes gt = g * t (bf16), the gate outputs and the
+//    mask count.  Nothing in it depends on y, so it can run concurrently with
+//    the EC-disabled GEMM (the semi-fused DAG).
+//  phase 2, B items (64 tokens, 32 output channels): gt . B' with MMA k-steps,
+//    scaled by s_n (per-channel fold), read-modify-write of y.
+// Stream order between the launches replaces any device-side wait: no item
+// waits for another, and the CTAs need not be co-resident.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -37,7 +32,6 @@ struct EcArgs {
   const __half* scales;
   float* part;       // [ksplit][Mpad][RT]
   int* tickets;      // [Mb16]
-  int* mflags;       // [Mb16]
   __nv_bfloat16* gt; // [Mpad][r]
   float* gate_out;
   int* mask_count;
@@ -46,7 +40,7 @@ struct EcArgs {
   float b_g, tau;
   int ksplit, RT, Mb16, Mpad, E;
   int itemsA, itemsB;
-  int phase;         // 0: both item kinds in one launch, 1: A items only, 2: B items only
+  int phase;         // 1: A items (projection and gate), 2: B items (update of y)
 };
 
 __device__ __forceinline__ uint32_t w8(const uint4& a, const uint4& b, int i) {
@@ -55,7 +49,7 @@ __device__ __forceinline__ uint32_t w8(const uint4& a, const uint4& b, int i) {
   return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
 }
 
-__device__ void ec_item_project(const EcArgs& a, int item, int lane, int epoch) {
+__device__ void ec_item_project(const EcArgs& a, int item, int lane) {
   const int mb = item / a.ksplit, ks = item % a.ksplit;
   const int KT = a.K / 64;
   const int kt0 = (int)((long long)ks * KT / a.ksplit), kt1 = (int)((long long)(ks + 1) * KT / a.ksplit);
@@ -139,36 +133,49 @@ __device__ void ec_item_project(const EcArgs& a, int item, int lane, int epoch) 
   const bool valid = lane < 16 && mb * 16 + lane < a.M;
   if (a.gate_out && valid) a.gate_out[mb * 16 + lane] = gm;
   const unsigned below = __ballot_sync(0xffffffffu, valid && gm < a.tau);
-  // every lane owns (token, column) pairs; K parts summed in order 0..ksplit-1
-  for (int idx = lane; idx < 16 * a.r; idx += 32) {
-    const int mm = idx / a.r, j = idx % a.r;
-    const int m = mb * 16 + mm;
-    const float* src = a.part + (size_t)m * a.RT + j;
-    const size_t stride = (size_t)a.Mpad * a.RT;
-    float t = 0.f;
-    int k2 = 0;
-    for (; k2 + 4 <= a.ksplit; k2 += 4) {
-      const float v0 = __ldcg(src + (k2 + 0) * stride), v1 = __ldcg(src + (k2 + 1) * stride);
-      const float v2 = __ldcg(src + (k2 + 2) * stride), v3 = __ldcg(src + (k2 + 3) * stride);
-      t += v0;
-      t += v1;
-      t += v2;
-      t += v3;
+  // every lane owns (token, 4 columns) groups; K parts summed in order
+  // 0..ksplit-1.  All parts of two groups are loaded before any sum, so a
+  // lane has up to 16 independent 16-byte loads in flight.
+  const int r4 = a.r / 4;
+  const size_t stride = (size_t)a.Mpad * a.RT;
+  for (int i0 = lane; i0 < 16 * r4; i0 += 64) {
+    float4 v[2][8];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int idx = i0 + 32 * u;
+      const int m = mb * 16 + idx / r4, j = 4 * (idx % r4);
+      const float* src = a.part + (size_t)m * a.RT + j;
+#pragma unroll
+      for (int k2 = 0; k2 < 8; ++k2)
+        if (idx < 16 * r4 && k2 < a.ksplit) v[u][k2] = __ldcg(reinterpret_cast<const float4*>(src + k2 * stride));
     }
-    for (; k2 < a.ksplit; ++k2) t += __ldcg(src + k2 * stride);
-    // the gate of token mm lives in lane mm; 16*r is a multiple of 32, so every
-    // lane runs the same number of iterations and the shuffle is convergent
-    const float g = __shfl_sync(0xffffffffu, gm, mm);
-    a.gt[(size_t)m * a.r + j] = __float2bfloat16_rn(g * t);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int idx = i0 + 32 * u;
+      // the gate of token mm lives in lane mm; every lane runs the shuffle
+      const int mm = (idx < 16 * r4 ? idx : 0) / r4;
+      const float g = __shfl_sync(0xffffffffu, gm, mm);
+      if (idx >= 16 * r4) continue;
+      const int m = mb * 16 + mm, j = 4 * (idx % r4);
+      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k2 = 0; k2 < 8; ++k2)
+        if (k2 < a.ksplit) {
+          t.x += v[u][k2].x;
+          t.y += v[u][k2].y;
+          t.z += v[u][k2].z;
+          t.w += v[u][k2].w;
+        }
+      uint2 o;
+      o.x = pack_bf16x2(g * t.x, g * t.y);
+      o.y = pack_bf16x2(g * t.z, g * t.w);
+      *reinterpret_cast<uint2*>(a.gt + (size_t)m * a.r + j) = o;
+    }
   }
   __syncwarp();
   if (lane == 0) {
     a.tickets[mb] = 0;
-    if (a.mask_count) atomicAdd(a.phase == 0 ? &a.hdr->ec_done : &a.hdr->sf_count, __popc(below));
-    if (a.phase == 0) {
-      __threadfence();
-      st_release_gpu(&a.mflags[mb], epoch + 1);
-    }
+    if (a.mask_count) atomicAdd(&a.hdr->sf_count, __popc(below));
   }
 }
 
@@ -213,17 +220,11 @@ __device__ __forceinline__ void ec_up_chunk(const EcArgs& a, int m0, int pair, i
   }
 }
 
-__device__ void ec_item_update(const EcArgs& a, int item, int lane, int epoch, __nv_bfloat16* stage) {
+__device__ void ec_item_update(const EcArgs& a, int item, int lane, __nv_bfloat16* stage) {
   const int P2 = a.N / 32;
   const int mb64 = item / P2, pair = item % P2;
   const int m0 = mb64 * 64;
   const int rho = lane >> 2, cq = lane & 3;
-  bool ok = true;
-  if (a.phase == 0 && lane < 4) {
-    const int mb = mb64 * 4 + lane;
-    if (mb < a.Mb16) ok = wait_flag_eq(&a.mflags[mb], epoch + 1, a.hdr);
-  }
-  ok = __all_sync(0xffffffffu, ok);
   float acc[2][8][4];
 #pragma unroll
   for (int si = 0; si < 2; ++si)
@@ -231,7 +232,7 @@ __device__ void ec_item_update(const EcArgs& a, int item, int lane, int epoch, _
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[si][nt][i] = 0.f;
-  if (ok) {
+  {
     if (a.r >= 64) {
       for (int jb = 0; jb < a.r; jb += 64) ec_up_chunk<4>(a, m0, pair, lane, jb, acc);
     } else if (a.r == 32) {
@@ -281,17 +282,11 @@ __device__ void ec_item_update(const EcArgs& a, int item, int lane, int epoch, _
 __global__ void __launch_bounds__(EC_WARPS * 32) ec_kernel(const __grid_constant__ EcArgs a) {
   __shared__ __align__(16) __nv_bfloat16 stage_all[EC_WARPS][64 * 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int epoch = *reinterpret_cast<volatile int*>(&a.hdr->epoch);
   const int gw = blockIdx.x * EC_WARPS + warp, nw = gridDim.x * EC_WARPS;
-  for (int it = gw; it < a.itemsA + a.itemsB; it += nw) {
-    if (it < a.itemsA)
-      ec_item_project(a, it, lane, epoch);
-    else
-      ec_item_update(a, it - a.itemsA, lane, epoch, stage_all[warp]);
-  }
-  if (a.phase == 2) return;
-  __syncthreads();
   if (a.phase == 1) {
+    for (int it = gw; it < a.itemsA; it += nw) ec_item_project(a, it, lane);
+    // the last CTA publishes the mask count of this launch
+    __syncthreads();
     if (threadIdx.x == 0 && a.mask_count) {
       __threadfence();
       const int prev = atomicAdd(&a.hdr->sf_done, 1);
@@ -302,18 +297,8 @@ __global__ void __launch_bounds__(EC_WARPS * 32) ec_kernel(const __grid_constant
         a.hdr->sf_count = 0;
       }
     }
-    return;
-  }
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const int prev = atomicAdd(&a.hdr->done_ctas, 1);
-    if (prev == (int)gridDim.x - 1) {
-      if (a.mask_count) *a.mask_count = a.hdr->ec_done;
-      a.hdr->done_ctas = 0;
-      a.hdr->ec_done = 0;
-      __threadfence();
-      atomicAdd(&a.hdr->epoch, 1);
-    }
+  } else {
+    for (int it = gw; it < a.itemsB; it += nw) ec_item_update(a, it, lane, stage_all[warp]);
   }
 }
 
@@ -335,8 +320,9 @@ EcPlan plan_ec(int M, int K, int N, int r, int sm_count) {
 }
 
 int launch_ec(const EcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, WsHeader* hdr,
-              float* part, int* tickets, int* mflags, __nv_bfloat16* gt, float* gate_out, int* mask_count,
-              cudaStream_t st, int phase) {
+              float* part, int* tickets, __nv_bfloat16* gt, float* gate_out, int* mask_count, cudaStream_t st,
+              int phase) {
+  if (phase != 1 && phase != 2) return set_error(SPEAR_ERR_INVALID_ARG, "EC launch phase must be 1 or 2");
   EcArgs a = {};
   a.x = x;
   a.y = y;
@@ -345,7 +331,6 @@ int launch_ec(const EcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
   a.scales = L.scales;
   a.part = part;
   a.tickets = tickets;
-  a.mflags = mflags;
   a.gt = gt;
   a.gate_out = gate_out;
   a.mask_count = mask_count;
@@ -362,26 +347,13 @@ int launch_ec(const EcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
   a.Mb16 = (M + 15) / 16;
   a.Mpad = ((M + 63) / 64) * 64;
   a.E = (L.r + 16) / 16;
-  a.itemsA = phase == 2 ? 0 : a.Mb16 * p.ksplit;
-  a.itemsB = phase == 1 ? 0 : (a.Mpad / 64) * (L.N / 32);
+  a.itemsA = a.Mb16 * p.ksplit;
+  a.itemsB = (a.Mpad / 64) * (L.N / 32);
   a.phase = phase;
-  // every CTA must be resident at once: B items wait for A items of other CTAs
-  static int per_sm = 0;
-  if (per_sm == 0) {
-    int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, ec_kernel, EC_WARPS * 32, 0) != cudaSuccess || nb < 1) nb = 1;
-    per_sm = nb;
-  }
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int grid = p.grid < per_sm * sms ? p.grid : per_sm * sms;
-  if (phase != 0) {
-    // split phases never wait on one another's CTAs: no residency cap, and
-    // no more CTAs than the items need
-    const int need = (a.itemsA + a.itemsB + EC_WARPS - 1) / EC_WARPS;
-    grid = need < p.grid ? need : p.grid;
-  }
+  // no more CTAs than the items of this phase need
+  const int items = phase == 1 ? a.itemsA : a.itemsB;
+  const int need = (items + EC_WARPS - 1) / EC_WARPS;
+  const int grid = need < p.grid ? need : p.grid;
   ec_kernel<<<grid, EC_WARPS * 32, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPEAR_OK : set_cuda_error("ec kernel launch", e);

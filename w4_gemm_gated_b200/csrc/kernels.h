@@ -59,18 +59,18 @@ int launch_decode2(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloa
                    float* gate_out, int* mask_count, bool ec_only, cudaStream_t st);
 
 // ---- standalone EC kernel (ec.cu): y += g * (x.A).B, in place ----
-// phase 0: one launch; 1: projection (gt, gate, mask count) only; 2: the
-// in-place update only, after a phase-1 launch that stream order completed
+// Two launches: phase 1 writes gt, the gate outputs and the mask count
+// (independent of y); phase 2 updates y, after phase 1 in stream order.
 struct EcPlan {
   int ksplit;   // K parts of the projection
-  int grid;     // persistent CTAs
+  int grid;     // CTAs at most
   int RT;       // row stride of projection partials
   size_t part_floats;  // floats of the partial buffer
 };
 EcPlan plan_ec(int M, int K, int N, int r, int sm_count);
 int launch_ec(const EcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y,
-              WsHeader* hdr, float* part, int* tickets, int* mflags, __nv_bfloat16* gt, float* gate_out,
-              int* mask_count, cudaStream_t st, int phase = 0);
+              WsHeader* hdr, float* part, int* tickets, __nv_bfloat16* gt, float* gate_out, int* mask_count,
+              cudaStream_t st, int phase);
 
 // ---- tensor-core path (tc_gemm.cu) ----
 struct TcPlan {
