@@ -30,6 +30,9 @@ Readings where the pages are silent (each also listed in the design doc):
   * the packed layout is the library's own (defined in ``pack_w4`` below and
     in the public header); the pages give none.
 
+The pages' own gate form, W + alpha B diag(gamma(A x)) A with gamma a
+bottleneck MLP, is ``linear_rank_gated`` below (per-rank gates).
+
 Parity status: every function here is pinned by ``tests/test_oracle.py``
 against hand-worked fixtures, closed forms, invariants or brute force.
 """
@@ -286,6 +289,87 @@ def linear_bruteforce(x_bits, q, s, group, A_bits, B_bits, w_g_bits, b_g):
                     e += t[j] * B[j, n]
                 acc += gm * e
             y[m, n] = acc
+    return y
+
+
+# ----------------------------------------------------------------------------
+# The pages' per-rank gate: gamma(t), a bottleneck MLP on t = x . A
+# ----------------------------------------------------------------------------
+
+def rank_gate(t: np.ndarray, W1: np.ndarray, b1: np.ndarray, W2: np.ndarray,
+              b2: np.ndarray) -> np.ndarray:
+    """gamma(t) = sigmoid(W2 . relu(W1 . t + b1) + b2), one row per token, float64.
+
+    SPEAR, gist.science technical summary, section 2.1 A: the effective weight
+    is W + alpha B diag(gamma(A x)) A with gamma "a bottleneck MLP" on the
+    low-rank projection.  The pages name neither the layers nor the
+    activation; this is the plainest reading: r -> h (ReLU) -> r (sigmoid, so
+    every rank's gate lies in (0, 1) like the scalar gate).
+    t: M x r; W1: h x r; b1: h; W2: r x h; b2: r (fp32 values, read exactly).
+    """
+    W1 = np.asarray(W1, dtype=np.float32).astype(np.float64)
+    W2 = np.asarray(W2, dtype=np.float32).astype(np.float64)
+    b1 = np.asarray(b1, dtype=np.float32).astype(np.float64)
+    b2 = np.asarray(b2, dtype=np.float32).astype(np.float64)
+    u = np.maximum(t @ W1.T + b1, 0.0)
+    z = u @ W2.T + b2
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-z))
+
+
+def linear_rank_gated(x_bits: np.ndarray, q: np.ndarray, s: np.ndarray, group: int,
+                      A_bits: np.ndarray, B_bits: np.ndarray, W1: np.ndarray, b1: np.ndarray,
+                      W2: np.ndarray, b2: np.ndarray, alpha: float
+                      ) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """y = x . dequant(W4) + alpha * ((x . A) * gamma(x . A)) . B, float64.
+
+    The row-vector form of W + alpha B diag(gamma(A x)) A (summary section
+    2.1 A).  Returns (y, gamma, gate_mean) with gate_mean[m] the mean over the
+    r ranks of gamma, the per-token gate this form reports (and compares with
+    tau for the mask count).
+    """
+    x = bf16_to_f64(x_bits)
+    y = x @ dequantize(q, s, group)
+    t = x @ bf16_to_f64(A_bits)
+    gam = rank_gate(t, W1, b1, W2, b2)
+    y = y + float(alpha) * ((t * gam) @ bf16_to_f64(B_bits))
+    return y, gam, gam.mean(axis=1)
+
+
+def linear_rank_gated_bruteforce(x_bits, q, s, group, A_bits, B_bits, W1, b1, W2, b2, alpha):
+    """Element-by-element loops over the same definition (tiny inputs only)."""
+    x = bf16_to_f64(x_bits)
+    A = bf16_to_f64(A_bits)
+    B = bf16_to_f64(B_bits)
+    W1 = np.asarray(W1, dtype=np.float32)
+    W2 = np.asarray(W2, dtype=np.float32)
+    b1 = np.asarray(b1, dtype=np.float32)
+    b2 = np.asarray(b2, dtype=np.float32)
+    s16 = np.asarray(s, dtype=np.float16)
+    M, K = x.shape
+    N = q.shape[0]
+    r = A.shape[1]
+    h = W1.shape[0]
+    y = np.zeros((M, N))
+    for m in range(M):
+        t = [sum(x[m, k] * A[k, j] for k in range(K)) for j in range(r)]
+        u = []
+        for i in range(h):
+            v = float(b1[i]) + sum(float(W1[i, j]) * t[j] for j in range(r))
+            u.append(v if v > 0.0 else 0.0)
+        gam = []
+        for j in range(r):
+            z = float(b2[j]) + sum(float(W2[j, i]) * u[i] for i in range(h))
+            gam.append(1.0 / (1.0 + math.exp(-z)) if z > -700 else 0.0)
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                sc = float(s16[n]) if group == 0 else float(s16[k // 128, n])
+                acc += x[m, k] * (sc * int(q[n, k]))
+            e = 0.0
+            for j in range(r):
+                e += t[j] * gam[j] * B[j, n]
+            y[m, n] = acc + float(alpha) * e
     return y
 
 

@@ -278,3 +278,88 @@ def test_synthetic_configs_shapes_and_gate_fraction():
     assert len(D.meta["outlier_channels"]) == 41
     g, _ = O.gate(D.x, D.w_g, D.b_g)
     assert g.shape == (16,) and np.all((g > 0) & (g < 1))
+
+
+# --------------------------------------------------------------------------
+# the pages' per-rank gate gamma(t) (bottleneck MLP on t = x . A)
+# --------------------------------------------------------------------------
+
+def _bits(v):
+    return O.f32_to_bf16_bits_rne(np.asarray(v, dtype=np.float32))
+
+
+def test_rank_gate_hand_worked():
+    # q = 0 (no W term), x = e_0, A row 0 = (1, 2): t = (1, 2).  h = 1:
+    # W1 . t + b1 = 0.5 - 2 + 2 = 0.5 -> relu 0.5; W2 . u + b2 = (1, -2);
+    # gamma = (sigmoid(1), sigmoid(-2)); B = (1, 1)^T, alpha = 0.5:
+    # y = 0.5 * (1 * sigmoid(1) + 2 * sigmoid(-2)).
+    K, N, r = 64, 1, 2
+    x = np.zeros((1, K), np.float32); x[0, 0] = 1.0
+    A = np.zeros((K, r), np.float32); A[0] = (1.0, 2.0)
+    B = np.ones((r, N), np.float32)
+    q = np.zeros((N, K), np.int8)
+    s = np.ones(N, np.float16)
+    W1 = np.array([[0.5, -1.0]], np.float32); b1 = np.array([2.0], np.float32)
+    W2 = np.array([[2.0], [-4.0]], np.float32); b2 = np.zeros(2, np.float32)
+    y, gam, gm = O.linear_rank_gated(_bits(x), q, s, 0, _bits(A), _bits(B), W1, b1, W2, b2, 0.5)
+    sig = lambda z: 1.0 / (1.0 + math.exp(-z))
+    assert y[0, 0] == pytest.approx(0.5 * (sig(1.0) + 2.0 * sig(-2.0)), rel=1e-15)
+    assert gam[0] == pytest.approx([sig(1.0), sig(-2.0)], rel=1e-15)
+    assert gm[0] == pytest.approx(0.5 * (sig(1.0) + sig(-2.0)), rel=1e-15)
+
+
+def _rank_case(seed, M=3, K=128, N=16, r=16, h=8, group=0):
+    rng = np.random.default_rng(seed)
+    x = _bits(rng.standard_normal((M, K)))
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    q, s = O.quantize_rtn(W, group)
+    A = _bits(rng.standard_normal((K, r)) * 0.05)
+    B = _bits(rng.standard_normal((r, N)) * 0.05)
+    W1 = (rng.standard_normal((h, r)) * 0.5).astype(np.float32)
+    b1 = (rng.standard_normal(h) * 0.1).astype(np.float32)
+    W2 = (rng.standard_normal((r, h)) * 0.5).astype(np.float32)
+    b2 = (rng.standard_normal(r) * 0.5).astype(np.float32)
+    return x, q, s, A, B, W1, b1, W2, b2
+
+
+@pytest.mark.parametrize("group", [0, 128])
+def test_rank_gated_matches_bruteforce(group):
+    x, q, s, A, B, W1, b1, W2, b2 = _rank_case(11 + group, K=256, group=group)
+    y, _, _ = O.linear_rank_gated(x, q, s, group, A, B, W1, b1, W2, b2, 0.75)
+    yb = O.linear_rank_gated_bruteforce(x, q, s, group, A, B, W1, b1, W2, b2, 0.75)
+    assert np.max(np.abs(y - yb)) <= 1e-12 * max(1.0, np.max(np.abs(yb)))
+
+
+def test_rank_gate_constant_reduces_to_scalar_gate():
+    # W1 = W2 = 0 and b2 = c on every rank: gamma = sigmoid(c) everywhere, which
+    # is the scalar gate with w_g = 0 and b_g = c (alpha = 1)
+    x, q, s, A, B, W1, b1, W2, b2 = _rank_case(21)
+    r, h = W2.shape
+    c = -0.7
+    y, gam, gm = O.linear_rank_gated(x, q, s, 0, A, B, np.zeros_like(W1), b1, np.zeros_like(W2),
+                                     np.full(r, c, np.float32), 1.0)
+    wg = _bits(np.zeros(x.shape[1]))
+    ys, g = O.linear(x, q, s, 0, A, B, wg, float(np.float32(c)))
+    assert np.allclose(y, ys, rtol=1e-13, atol=1e-15)
+    assert np.allclose(gm, g, rtol=1e-15)
+
+
+def test_rank_gate_off_gives_pure_w4_gemm():
+    x, q, s, A, B, W1, b1, W2, b2 = _rank_case(31)
+    y0, _ = O.linear(x, q, s, 0, None, None, None, 0.0)
+    ya, _, _ = O.linear_rank_gated(x, q, s, 0, A, B, W1, b1, W2, b2, 0.0)        # alpha = 0
+    yb, gam, _ = O.linear_rank_gated(x, q, s, 0, A, B, W1, b1, W2,
+                                     np.full(W2.shape[0], -1000.0, np.float32), 1.0)  # gamma -> 0
+    assert np.array_equal(ya, y0)
+    assert np.max(gam) < 1e-300
+    assert np.allclose(yb, y0, rtol=0, atol=1e-250)
+
+
+def test_rank_gate_relu_cuts_w1():
+    # b1 far below zero: relu gives u = 0 whatever W1 is, so gamma = sigmoid(b2)
+    x, q, s, A, B, W1, b1, W2, b2 = _rank_case(41)
+    t = O.bf16_to_f64(x) @ O.bf16_to_f64(A)
+    g1 = O.rank_gate(t, W1, np.full_like(b1, -1e6), W2, b2)
+    g2 = O.rank_gate(t, 3.0 * W1 + 1.0, np.full_like(b1, -1e6), W2, b2)
+    assert np.array_equal(g1, g2)
+    assert np.allclose(g1, expit(b2.astype(np.float64))[None, :], rtol=1e-15)
