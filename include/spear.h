@@ -152,9 +152,30 @@ typedef struct spear_layer {
   const uint16_t* scales;  /* device fp16, spear_scale_count(N, K, group) values  */
   const uint16_t* AgT;     /* device bf16 (r+1) x K from spear_ec_pack (r > 0)    */
   const uint16_t* BpT;     /* device bf16 N x r from spear_ec_pack (r > 0)        */
-  float b_g;               /* gate bias                                           */
+  float b_g;               /* gate bias (scalar gate)                             */
   float gate_tau;          /* threshold of the gate-mask count; <= 0 means 0.1    */
+  /* Gate form.  A zero-initialised tail keeps the scalar gate.
+   * SPEAR_GATE_RANK_MLP is the pages' form (gist.science technical summary,
+   * section 2.1 A: effective weight W + alpha B diag(gamma(A x)) A, gamma a
+   * bottleneck MLP on the low-rank projection):
+   *   t = x . A,  u = relu(W1 t + b1),  gamma = sigmoid(W2 u + b2),
+   *   y = x . dequant(W4) + alpha * (t * gamma) . B,
+   * with gt = bf16(alpha * gamma * t) feeding the up-projection.  The row of
+   * w_g in AgT is then unused (pack it with w_g = 0); b_g is ignored.  The
+   * per-token gate reported by gate_out (and compared with gate_tau) is the
+   * mean of gamma over the r ranks.  Paths: the decode kernel (not its
+   * fallback for K % 256 != 0 or very long K), the tensor-core kernel, and
+   * the unfused / semi-fused EC kernel. */
+  int gate_kind;           /* SPEAR_GATE_SCALAR (0) or SPEAR_GATE_RANK_MLP (1)    */
+  int gate_hidden;         /* h, the bottleneck width of the rank gate: 8, 16, 32 */
+  const float* gate_w1;    /* device fp32 h x r row-major (16-byte aligned)       */
+  const float* gate_b1;    /* device fp32 [h]                                     */
+  const float* gate_w2;    /* device fp32 r x h row-major                         */
+  const float* gate_b2;    /* device fp32 [r]                                     */
+  float gate_alpha;        /* alpha of the rank gate                              */
 } spear_layer;
+
+enum { SPEAR_GATE_SCALAR = 0, SPEAR_GATE_RANK_MLP = 1 };
 
 /* Workspace bytes needed by spear_linear_forward* for any 1 <= M <= M_max
  * (0 on invalid arguments).  The workspace holds split-K partials, the EC

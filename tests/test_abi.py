@@ -206,3 +206,22 @@ def test_slo_chunk_matches_enumeration(S):
     with pytest.raises(S.SpearError):
         S.slo_chunk(layers, 1, 100.0, [-4])
     S.dispatch_clear()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(gate_kind=2), 1),
+    (dict(gate_kind=1, r=0), 1),
+    (dict(gate_kind=1, gate_hidden=12), 2),
+    (dict(gate_kind=1, gate_hidden=16, gate_w2=None), 1),
+    (dict(gate_kind=1, gate_hidden=16, gate_b1=0x8004), 3),
+])
+def test_rank_gate_validation_before_launch(S, kw, code):
+    d = dict(gate_kind=0, gate_hidden=0, gate_w1=0x80000, gate_b1=0x81000, gate_w2=0x82000, gate_b2=0x83000,
+             gate_alpha=1.0)
+    d.update(kw)
+    st = _layer(S, **{k: v for k, v in kw.items() if k == "r"})
+    for k in ("gate_kind", "gate_hidden", "gate_w1", "gate_b1", "gate_w2", "gate_b2", "gate_alpha"):
+        setattr(st, k, d[k])
+    rc = S.F["spear_linear_forward"](ctypes.byref(st), 0x50000, 4, 0x60000, 0x70000, 1 << 30, None, None, None)
+    assert rc == code, S.F["spear_last_error"]().decode()
+    assert S.F["spear_last_error"]().decode()

@@ -83,6 +83,27 @@ static int check_layer(const spear_layer* l, LayerView* out) {
   out->bpt = l->r > 0 ? reinterpret_cast<const __nv_bfloat16*>(l->BpT) : nullptr;
   out->b_g = l->b_g;
   out->tau = l->gate_tau > 0.f ? l->gate_tau : 0.1f;
+  out->gate_kind = l->gate_kind;
+  out->gate_h = 0;
+  out->gw1 = out->gb1 = out->gw2 = out->gb2 = nullptr;
+  out->alpha = 1.f;
+  if (l->gate_kind != SPEAR_GATE_SCALAR && l->gate_kind != SPEAR_GATE_RANK_MLP)
+    return set_error(SPEAR_ERR_INVALID_ARG, "gate_kind=%d: must be 0 (scalar) or 1 (rank MLP)", l->gate_kind);
+  if (l->gate_kind == SPEAR_GATE_RANK_MLP) {
+    if (l->r == 0) return set_error(SPEAR_ERR_INVALID_ARG, "the rank gate needs an EC (r > 0)");
+    if (l->gate_hidden != 8 && l->gate_hidden != 16 && l->gate_hidden != 32)
+      return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "gate_hidden=%d: must be 8, 16 or 32", l->gate_hidden);
+    if (!l->gate_w1 || !l->gate_b1 || !l->gate_w2 || !l->gate_b2)
+      return set_error(SPEAR_ERR_INVALID_ARG, "the rank gate needs gate_w1, gate_b1, gate_w2 and gate_b2");
+    if (!aligned16(l->gate_w1) || !aligned16(l->gate_b1) || !aligned16(l->gate_w2) || !aligned16(l->gate_b2))
+      return set_error(SPEAR_ERR_ALIGNMENT, "rank-gate parameters must be 16-byte aligned");
+    out->gate_h = l->gate_hidden;
+    out->gw1 = l->gate_w1;
+    out->gb1 = l->gate_b1;
+    out->gw2 = l->gate_w2;
+    out->gb2 = l->gate_b2;
+    out->alpha = l->gate_alpha;
+  }
   return SPEAR_OK;
 }
 
@@ -231,8 +252,11 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
   const int sms = sm_count();
   if (path == SPEAR_PATH_DECODE) {
     if (M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs M <= 16 (M=%d)", M);
-    if (!decode2_unsupported(M, L.K, L.N, L.r))
+    if (!decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind))
       return launch_decode2(L, x, M, y, hdr, tbuf, gate_out, mask_count, false, st);
+    if (L.gate_kind)
+      return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: the rank gate needs the main decode kernel (%s)",
+                       decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind));
     DecodePlan p = plan_decode(M, L.K, L.N, L.r, L.group, sms);
     const char* why = check_decode_plan(p);
     if (why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", why);
@@ -243,14 +267,17 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
     L0.r = 0;
     L0.agt = nullptr;
     L0.bpt = nullptr;
+    L0.gate_kind = 0;
     int rc;
-    if (M <= 16 && !decode2_unsupported(M, L.K, L.N, L.r)) {
+    if (M <= 16 && !decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind)) {
       rc = launch_decode2(L0, x, M, y, hdr, tbuf, L.r > 0 ? nullptr : gate_out, L.r > 0 ? nullptr : mask_count,
                           false, st);
       if (rc || L.r == 0) return rc;
       // the separate EC launch: same kernel in EC-only mode, y += g (t . B) in place
       return launch_decode2(L, x, M, y, hdr, tbuf, gate_out, mask_count, true, st);
     } else if (M <= 16) {
+      if (L.gate_kind)
+        return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "unfused path at M <= 16: the rank gate needs the main decode kernel");
       DecodePlan p = plan_decode(M, L.K, L.N, 0, L.group, sms);
       const char* why = check_decode_plan(p);
       if (why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", why);
@@ -279,7 +306,8 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
     L0.r = 0;
     L0.agt = nullptr;
     L0.bpt = nullptr;
-    const bool d2 = M <= 16 && !decode2_unsupported(M, L.K, L.N, L.r);
+    L0.gate_kind = 0;
+    const bool d2 = M <= 16 && !decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind);
     auto gemm = [&](float* go, int* mc) {
       if (d2) return launch_decode2(L0, x, M, y, hdr, tbuf, go, mc, false, st);
       TcPlan p = plan_tc(M, L.K, L.N, 0, L.group, sms);

@@ -85,15 +85,19 @@ struct D2Args {
   int ES;                   // EC strips (0: EC off)
   int nslot, own_cap;
   int ec_only;              // 1: no weights, y += EC term in place (unfused path)
+  int gate_kind, gate_h;    // 0: scalar gate; 1: per-rank gamma(t) with bottleneck h
+  const float *gw1, *gb1, *gw2, *gb2;
+  float alpha;
   short4 cl_tab[D2_MAXCL];  // per cluster: first EC strip, EC strips, first weight strip, weight strips
 };
 
 // Shared-memory carve-up (same on host and device).
 struct D2Smem {
-  uint32_t ring, red, recv, park, bps, scs, ts, gts, stage, bars, total;
+  uint32_t ring, red, recv, park, bps, scs, ts, gts, gsc, stage, bars, total;
 };
 __host__ __device__ __forceinline__ uint32_t d2_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
-__host__ __device__ __forceinline__ D2Smem d2_smem(int MT, int nslot, int CS, int own_cap, int r, int ES) {
+__host__ __device__ __forceinline__ D2Smem d2_smem(int MT, int nslot, int CS, int own_cap, int r, int ES,
+                                                   int gate_kind) {
   D2Smem s;
   const uint32_t NT = MT / 8;
   uint32_t off = 0;
@@ -113,6 +117,8 @@ __host__ __device__ __forceinline__ D2Smem d2_smem(int MT, int nslot, int CS, in
   off += ES * MT * 16 * 8;
   s.gts = off;  // gt [MT][r + 8] bf16
   off += d2_up(MT * (r + 8) * 2, 16);
+  s.gsc = off;  // rank gate: hidden activations [MT][32] fp32
+  off += gate_kind ? MT * 32 * 4 : 0;
   s.stage = off;
   off += MT * 32;
   s.bars = off;
@@ -325,29 +331,93 @@ __device__ __forceinline__ void d2_ts_fetch(const unsigned long long* tt, unsign
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Gate and gt from the staged projection (one warp): g_m = sigmoid(t[m][r] + b_g),
-// gt[m][j] = bf16(g_m t[m][j]); CTA 0 also writes the gate outputs.
+// Gate and gt from the staged projection (one warp).  Scalar gate:
+// g_m = sigmoid(t[m][r] + b_g), gt[m][j] = bf16(g_m t[m][j]).  Rank gate
+// (summary section 2.1 A): u = relu(W1 t + b1), gamma = sigmoid(W2 u + b2),
+// gt[m][j] = bf16(alpha gamma_j t[m][j]), and the reported gate is the mean of
+// gamma.  CTA 0 also writes the gate outputs and the mask count.
 template <int MT>
-__device__ void d2_build_gt(const D2Args& a, const unsigned long long* ts, __nv_bfloat16* gts, int lane) {
+__device__ void d2_build_gt(const D2Args& a, const unsigned long long* ts, __nv_bfloat16* gts, float* gsc, int lane) {
   auto tval = [&](int m, int row) {
     return __uint_as_float((uint32_t)ts[((row >> 4) * MT + m) * 16 + (row & 15)]);
   };
-  const float g = lane < MT ? sigmoidf_(tval(lane, a.r) + a.b_g) : 0.f;
+  const int gs = a.r + 8;
+  float g;  // lane m: token m's gate
+  if (a.gate_kind == 1) {
+    const int h = a.gate_h, r = a.r;
+    // hidden activations of the live tokens
+    for (int idx = lane; idx < MT * h; idx += 32) {
+      const int m = idx / h, i = idx - m * h;
+      float v = 0.f;
+      if (m < a.M) {
+        v = __ldg(a.gb1 + i);
+        const float4* w = reinterpret_cast<const float4*>(a.gw1 + (size_t)i * r);
+        for (int j4 = 0; j4 < r / 4; ++j4) {
+          const float4 wv = __ldg(w + j4);
+          v = fmaf(wv.x, tval(m, 4 * j4), v);
+          v = fmaf(wv.y, tval(m, 4 * j4 + 1), v);
+          v = fmaf(wv.z, tval(m, 4 * j4 + 2), v);
+          v = fmaf(wv.w, tval(m, 4 * j4 + 3), v);
+        }
+        v = fmaxf(v, 0.f);
+      }
+      gsc[m * 32 + i] = v;
+    }
+    __syncwarp();
+    // gamma and gt by (token, rank); MT * r is a multiple of 32, and a batch of
+    // 32 pairs holds one token (r >= 32) or two (r = 16)
+    float gsum = 0.f;
+    for (int base = 0; base < MT * r; base += 32) {
+      const int idx = base + lane;
+      const int m = idx / r, j = idx - m * r;
+      float gam = 0.f, o = 0.f;
+      if (m < a.M) {
+        float z = __ldg(a.gb2 + j);
+        const float4* w = reinterpret_cast<const float4*>(a.gw2 + (size_t)j * h);
+        for (int i4 = 0; i4 < h / 4; ++i4) {
+          const float4 wv = __ldg(w + i4);
+          z = fmaf(wv.x, gsc[m * 32 + 4 * i4], z);
+          z = fmaf(wv.y, gsc[m * 32 + 4 * i4 + 1], z);
+          z = fmaf(wv.z, gsc[m * 32 + 4 * i4 + 2], z);
+          z = fmaf(wv.w, gsc[m * 32 + 4 * i4 + 3], z);
+        }
+        gam = sigmoidf_(z);
+        o = a.alpha * gam * tval(m, j);
+      }
+      gts[m * gs + j] = __float2bfloat16_rn(o);
+      // this batch's gamma sum per token, by a fixed shuffle tree
+      float v = gam;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1)
+        if (off < r) v += __shfl_xor_sync(0xffffffffu, v, off);
+      const int m0 = base / r;
+      if (r >= 32) {
+        if (lane == m0) gsum += v;
+      } else {
+        const float v0 = __shfl_sync(0xffffffffu, v, 0), v1 = __shfl_sync(0xffffffffu, v, 16);
+        if (lane == m0) gsum += v0;
+        if (lane == m0 + 1) gsum += v1;
+      }
+    }
+    g = gsum / (float)r;
+  } else {
+    g = lane < MT ? sigmoidf_(tval(lane, a.r) + a.b_g) : 0.f;
+    const int half = a.r / 2;
+    for (int base = 0; base < MT * half; base += 32) {
+      const int idx = base + lane;
+      const int m = idx / half;
+      const float gm = __shfl_sync(0xffffffffu, g, m < MT ? m : 0);
+      if (idx < MT * half) {
+        const int j = 2 * (idx - m * half);
+        *reinterpret_cast<uint32_t*>(gts + m * gs + j) = pack_bf16x2(gm * tval(m, j), gm * tval(m, j + 1));
+      }
+    }
+  }
   if (blockIdx.x == 0) {
     const bool valid = lane < a.M;
     if (a.gate_out && valid) a.gate_out[lane] = g;
     const unsigned below = __ballot_sync(0xffffffffu, valid && g < a.tau);
     if (a.mask_count && lane == 0) *a.mask_count = __popc(below);
-  }
-  const int gs = a.r + 8, half = a.r / 2;
-  for (int base = 0; base < MT * half; base += 32) {
-    const int idx = base + lane;
-    const int m = idx / half;
-    const float gm = __shfl_sync(0xffffffffu, g, m < MT ? m : 0);
-    if (idx < MT * half) {
-      const int j = 2 * (idx - m * half);
-      *reinterpret_cast<uint32_t*>(gts + m * gs + j) = pack_bf16x2(gm * tval(m, j), gm * tval(m, j + 1));
-    }
   }
   __syncwarp();
 }
@@ -367,7 +437,7 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
   // 1024-byte aligned base, derived from the shared array itself so that the
   // compiler keeps every access in the shared window (ld/st.shared)
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const D2Smem SL = d2_smem(MT, a.nslot, a.CS, a.own_cap, a.r, a.ES);
+  const D2Smem SL = d2_smem(MT, a.nslot, a.CS, a.own_cap, a.r, a.ES, a.gate_kind);
   uint8_t* ring = sm + SL.ring;
   float4* red = reinterpret_cast<float4*>(sm + SL.red);
   float4* recv = reinterpret_cast<float4*>(sm + SL.recv);
@@ -376,6 +446,7 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
   __half* scs = reinterpret_cast<__half*>(sm + SL.scs);
   unsigned long long* ts = reinterpret_cast<unsigned long long*>(sm + SL.ts);
   __nv_bfloat16* gts = reinterpret_cast<__nv_bfloat16*>(sm + SL.gts);
+  float* gsc = reinterpret_cast<float*>(sm + SL.gsc);
   __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sm + SL.stage);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + SL.bars);
   uint64_t* empty = full + a.nslot;
@@ -704,7 +775,7 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
         }
         tok = __all_sync(FULL, tok);
         if (tok && gst == 2) {
-          d2_build_gt<MT>(a, ts, gts, lane);
+          d2_build_gt<MT>(a, ts, gts, gsc, lane);
           gst = 3;
           // every CTA reads the projection once; the last reader advances the epoch
           if (lane == 0) obs_prev = atomicAdd(&a.hdr->gt_obs, 1);
@@ -933,8 +1004,10 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
       }
     }
   }
-  // no CTA of the cluster leaves while st.async writes into it may be in flight
-  if (a.CS > 1) cluster_sync_all();
+  // no CTA of the cluster leaves while st.async writes into it may be in flight.
+  // Lifetime only: nothing is read after the barrier, so the arrival is relaxed
+  // and does not wait for this thread's global stores (a release would).
+  if (a.CS > 1) asm volatile("barrier.cluster.arrive.relaxed;\n\tbarrier.cluster.wait;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -964,7 +1037,7 @@ static cudaError_t d2_attrs(size_t smem) {
   return cudaSuccess;
 }
 
-static D2Plan make_d2_plan(int MT, int K, int N, int r, int sms) {
+static D2Plan make_d2_plan(int MT, int K, int N, int r, int sms, int gate_kind) {
   D2Plan p = {};
   p.MT = MT;
   p.why = nullptr;
@@ -1021,26 +1094,26 @@ static D2Plan make_d2_plan(int MT, int K, int N, int r, int sms) {
     p.why = "too many strips per CTA for the decode kernel";
     return p;
   }
-  const D2Smem s0 = d2_smem(MT, 0, p.CS, own, r, p.ES);
+  const D2Smem s0 = d2_smem(MT, 0, p.CS, own, r, p.ES, gate_kind);
   const size_t per_slot = D2_SLOT + 16;
   p.nslot = (int)std::min<size_t>(D2_MAXSLOT, (D2_SMEM_CAP - std::min<size_t>(s0.total, D2_SMEM_CAP)) / per_slot);
   if (p.nslot < 3) {
     p.why = "shared memory too small for the decode kernel's ring";
     return p;
   }
-  p.smem = d2_smem(MT, p.nslot, p.CS, own, r, p.ES).total;
+  p.smem = d2_smem(MT, p.nslot, p.CS, own, r, p.ES, gate_kind).total;
   return p;
 }
 
-static const D2Plan& d2_plan(int MT, int K, int N, int r, int sms) {
+static const D2Plan& d2_plan(int MT, int K, int N, int r, int sms, int gate_kind) {
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int, int, int, int>, D2Plan> cache;
+  static std::map<std::tuple<int, int, int, int, int, int, int>, D2Plan> cache;
   int dev = 0;
   cudaGetDevice(&dev);
-  const auto key = std::make_tuple(dev, MT, K, N, r, sms);
+  const auto key = std::make_tuple(dev, MT, K, N, r, sms, gate_kind);
   std::lock_guard<std::mutex> lk(mu);
   auto it = cache.find(key);
-  if (it == cache.end()) it = cache.emplace(key, make_d2_plan(MT, K, N, r, sms)).first;
+  if (it == cache.end()) it = cache.emplace(key, make_d2_plan(MT, K, N, r, sms, gate_kind)).first;
   return it->second;
 }
 
@@ -1049,9 +1122,9 @@ size_t decode2_tt_bytes(int r) {
   return (size_t)ES * 16 * 16 * 8;
 }
 
-const char* decode2_unsupported(int M, int K, int N, int r) {
+const char* decode2_unsupported(int M, int K, int N, int r, int gate_kind) {
   if (M < 1 || M > 16) return "the decode kernel needs 1 <= M <= 16";
-  return d2_plan(M <= 8 ? 8 : 16, K, N, r, device_sm_count()).why;
+  return d2_plan(M <= 8 ? 8 : 16, K, N, r, device_sm_count(), gate_kind).why;
 }
 
 template <int MT, int KTW, bool GROUP>
@@ -1108,7 +1181,8 @@ int launch_decode2(const LayerView& Lv, const __nv_bfloat16* x, int M, __nv_bflo
                    float* gate_out, int* mask_count, bool ec_only, cudaStream_t st) {
   if (M < 1 || M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs 1 <= M <= 16 (M=%d)", M);
   const int MT = M <= 8 ? 8 : 16;
-  const D2Plan& p = d2_plan(MT, Lv.K, Lv.N, Lv.r, device_sm_count());
+  const int gk = Lv.r > 0 ? Lv.gate_kind : 0;
+  const D2Plan& p = d2_plan(MT, Lv.K, Lv.N, Lv.r, device_sm_count(), gk);
   if (p.why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", p.why);
   if (ec_only && Lv.r == 0) return set_error(SPEAR_ERR_INVALID_ARG, "EC-only launch without an EC");
   D2Args a = {};
@@ -1134,6 +1208,13 @@ int launch_decode2(const LayerView& Lv, const __nv_bfloat16* x, int M, __nv_bflo
   a.nslot = p.nslot;
   a.own_cap = p.own_cap;
   a.ec_only = ec_only ? 1 : 0;
+  a.gate_kind = gk;
+  a.gate_h = Lv.gate_h;
+  a.gw1 = Lv.gw1;
+  a.gb1 = Lv.gb1;
+  a.gw2 = Lv.gw2;
+  a.gb2 = Lv.gb2;
+  a.alpha = Lv.alpha;
   for (int c = 0; c < p.NC; ++c) a.cl_tab[c] = p.cl_tab[c];
   CUtensorMap maps[3];
   memset(maps, 0, sizeof(maps));

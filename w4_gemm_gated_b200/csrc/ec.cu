@@ -41,6 +41,9 @@ struct EcArgs {
   int ksplit, RT, Mb16, Mpad, E;
   int itemsA, itemsB;
   int phase;         // 1: A items (projection and gate), 2: B items (update of y)
+  int gate_kind, gate_h;  // 0: scalar gate; 1: per-rank gamma(t) with bottleneck h
+  const float *gw1, *gb1, *gw2, *gb2;
+  float alpha;
 };
 
 __device__ __forceinline__ uint32_t w8(const uint4& a, const uint4& b, int i) {
@@ -123,16 +126,14 @@ __device__ void ec_item_project(const EcArgs& a, int item, int lane) {
   if (prev != a.ksplit - 1) return;
   __threadfence();
   // last K part of this m-block: fixed-order sums, gate, gt
+  const bool rank = a.gate_kind == 1;
   float gm = 0.f;
-  if (lane < 16) {
+  if (!rank && lane < 16) {
     const int m = mb * 16 + lane;
     float l = 0.f;
     for (int k2 = 0; k2 < a.ksplit; ++k2) l += __ldcg(a.part + ((size_t)k2 * a.Mpad + m) * a.RT + a.r);
     gm = sigmoidf_(l + a.b_g);
   }
-  const bool valid = lane < 16 && mb * 16 + lane < a.M;
-  if (a.gate_out && valid) a.gate_out[mb * 16 + lane] = gm;
-  const unsigned below = __ballot_sync(0xffffffffu, valid && gm < a.tau);
   // every lane owns (token, 4 columns) groups; K parts summed in order
   // 0..ksplit-1.  All parts of two groups are loaded before any sum, so a
   // lane has up to 16 independent 16-byte loads in flight.
@@ -166,12 +167,75 @@ __device__ void ec_item_project(const EcArgs& a, int item, int lane) {
           t.z += v[u][k2].z;
           t.w += v[u][k2].w;
         }
-      uint2 o;
-      o.x = pack_bf16x2(g * t.x, g * t.y);
-      o.y = pack_bf16x2(g * t.z, g * t.w);
-      *reinterpret_cast<uint2*>(a.gt + (size_t)m * a.r + j) = o;
+      if (rank) {
+        // the rank gate needs whole rows of t: keep the sum in part 0's slot
+        *reinterpret_cast<float4*>(a.part + (size_t)m * a.RT + j) = t;
+      } else {
+        uint2 o;
+        o.x = pack_bf16x2(g * t.x, g * t.y);
+        o.y = pack_bf16x2(g * t.z, g * t.w);
+        *reinterpret_cast<uint2*>(a.gt + (size_t)m * a.r + j) = o;
+      }
     }
   }
+  if (rank) {
+    // rank gate (summary section 2.1 A), one token per lane: u = relu(W1 t + b1),
+    // gamma = sigmoid(W2 u + b2), gt = bf16(alpha gamma t); the gate is mean(gamma)
+    __syncwarp();
+    __threadfence_block();
+    if (lane < 16) {
+      const int m = mb * 16 + lane, h = a.gate_h;
+      const float* trow = a.part + (size_t)m * a.RT;
+      float u[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) u[i] = i < h ? __ldg(a.gb1 + i) : 0.f;
+      for (int j = 0; j < a.r; j += 4) {
+        const float4 tv = __ldcg(reinterpret_cast<const float4*>(trow + j));
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (i < h) {
+            const float4 wv = __ldg(reinterpret_cast<const float4*>(a.gw1 + (size_t)i * a.r + j));
+            u[i] = fmaf(wv.x, tv.x, u[i]);
+            u[i] = fmaf(wv.y, tv.y, u[i]);
+            u[i] = fmaf(wv.z, tv.z, u[i]);
+            u[i] = fmaf(wv.w, tv.w, u[i]);
+          }
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) u[i] = fmaxf(u[i], 0.f);
+      float gsum = 0.f;
+      for (int j = 0; j < a.r; j += 4) {
+        const float4 tv = __ldcg(reinterpret_cast<const float4*>(trow + j));
+        const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
+        float o[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          float z = __ldg(a.gb2 + j + jj);
+          const float4* w = reinterpret_cast<const float4*>(a.gw2 + (size_t)(j + jj) * h);
+#pragma unroll
+          for (int i4 = 0; i4 < 8; ++i4)
+            if (4 * i4 < h) {
+              const float4 wv = __ldg(w + i4);
+              z = fmaf(wv.x, u[4 * i4], z);
+              z = fmaf(wv.y, u[4 * i4 + 1], z);
+              z = fmaf(wv.z, u[4 * i4 + 2], z);
+              z = fmaf(wv.w, u[4 * i4 + 3], z);
+            }
+          const float gam = sigmoidf_(z);
+          gsum += gam;
+          o[jj] = a.alpha * gam * tt[jj];
+        }
+        uint2 ov;
+        ov.x = pack_bf16x2(o[0], o[1]);
+        ov.y = pack_bf16x2(o[2], o[3]);
+        *reinterpret_cast<uint2*>(a.gt + (size_t)m * a.r + j) = ov;
+      }
+      gm = gsum / (float)a.r;
+    }
+  }
+  const bool valid = lane < 16 && mb * 16 + lane < a.M;
+  if (a.gate_out && valid) a.gate_out[mb * 16 + lane] = gm;
+  const unsigned below = __ballot_sync(0xffffffffu, valid && gm < a.tau);
   __syncwarp();
   if (lane == 0) {
     a.tickets[mb] = 0;
@@ -279,27 +343,31 @@ __device__ void ec_item_update(const EcArgs& a, int item, int lane, __nv_bfloat1
   __syncwarp();
 }
 
-__global__ void __launch_bounds__(EC_WARPS * 32) ec_kernel(const __grid_constant__ EcArgs a) {
+// Phase 1 and phase 2 are separate kernels, so the update keeps its own
+// (smaller) register allocation.
+__global__ void __launch_bounds__(EC_WARPS * 32) ec_project_kernel(const __grid_constant__ EcArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * EC_WARPS + warp, nw = gridDim.x * EC_WARPS;
+  for (int it = gw; it < a.itemsA; it += nw) ec_item_project(a, it, lane);
+  // the last CTA publishes the mask count of this launch
+  __syncthreads();
+  if (threadIdx.x == 0 && a.mask_count) {
+    __threadfence();
+    const int prev = atomicAdd(&a.hdr->sf_done, 1);
+    if (prev == (int)gridDim.x - 1) {
+      __threadfence();
+      *a.mask_count = *reinterpret_cast<volatile int*>(&a.hdr->sf_count);
+      a.hdr->sf_done = 0;
+      a.hdr->sf_count = 0;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(EC_WARPS * 32) ec_update_kernel(const __grid_constant__ EcArgs a) {
   __shared__ __align__(16) __nv_bfloat16 stage_all[EC_WARPS][64 * 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gw = blockIdx.x * EC_WARPS + warp, nw = gridDim.x * EC_WARPS;
-  if (a.phase == 1) {
-    for (int it = gw; it < a.itemsA; it += nw) ec_item_project(a, it, lane);
-    // the last CTA publishes the mask count of this launch
-    __syncthreads();
-    if (threadIdx.x == 0 && a.mask_count) {
-      __threadfence();
-      const int prev = atomicAdd(&a.hdr->sf_done, 1);
-      if (prev == (int)gridDim.x - 1) {
-        __threadfence();
-        *a.mask_count = *reinterpret_cast<volatile int*>(&a.hdr->sf_count);
-        a.hdr->sf_done = 0;
-        a.hdr->sf_count = 0;
-      }
-    }
-  } else {
-    for (int it = gw; it < a.itemsB; it += nw) ec_item_update(a, it, lane, stage_all[warp]);
-  }
+  for (int it = gw; it < a.itemsB; it += nw) ec_item_update(a, it, lane, stage_all[warp]);
 }
 
 EcPlan plan_ec(int M, int K, int N, int r, int sm_count) {
@@ -350,11 +418,21 @@ int launch_ec(const EcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
   a.itemsA = a.Mb16 * p.ksplit;
   a.itemsB = (a.Mpad / 64) * (L.N / 32);
   a.phase = phase;
+  a.gate_kind = L.gate_kind;
+  a.gate_h = L.gate_h;
+  a.gw1 = L.gw1;
+  a.gb1 = L.gb1;
+  a.gw2 = L.gw2;
+  a.gb2 = L.gb2;
+  a.alpha = L.alpha;
   // no more CTAs than the items of this phase need
   const int items = phase == 1 ? a.itemsA : a.itemsB;
   const int need = (items + EC_WARPS - 1) / EC_WARPS;
   const int grid = need < p.grid ? need : p.grid;
-  ec_kernel<<<grid, EC_WARPS * 32, 0, st>>>(a);
+  if (phase == 1)
+    ec_project_kernel<<<grid, EC_WARPS * 32, 0, st>>>(a);
+  else
+    ec_update_kernel<<<grid, EC_WARPS * 32, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPEAR_OK : set_cuda_error("ec kernel launch", e);
 }

@@ -30,6 +30,10 @@ struct LayerView {
   const __nv_bfloat16* agt;  // (r+1) x K, or null when r == 0
   const __nv_bfloat16* bpt;  // N x r, or null when r == 0
   float b_g, tau;
+  // gate form: 0 scalar sigmoid(x.w_g + b_g); 1 per-rank gamma(t) = sigmoid(W2 relu(W1 t + b1) + b2)
+  int gate_kind, gate_h;
+  const float *gw1, *gb1, *gw2, *gb2;  // h x r, h, r x h, r (kind 1)
+  float alpha;
 };
 
 // ---- decode path (decode.cu) ----
@@ -52,7 +56,7 @@ int launch_decode(const DecodePlan& p, const LayerView& L, const __nv_bfloat16* 
 
 // ---- decode path for back-to-back launches (decode2.cu) ----
 // null if the kernel can run (M, K, N, r), else the reason
-const char* decode2_unsupported(int M, int K, int N, int r);
+const char* decode2_unsupported(int M, int K, int N, int r, int gate_kind);
 // bytes of tagged EC projection words the kernel needs in the workspace
 size_t decode2_tt_bytes(int r);
 int launch_decode2(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, WsHeader* hdr, void* tt,

@@ -63,6 +63,9 @@ struct TcArgs {
   int with_ec;      // projection tiles + EC k-steps
   int NE;           // projection tile width: 16 * ceil((r + 1) / 16)
   int ec_steps;     // ceil(r / 64)
+  int gate_kind, gate_h;  // 0: scalar gate; 1: per-rank gamma(t) with bottleneck h
+  const float *gw1, *gb1, *gw2, *gb2;
+  float alpha;
 };
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -348,24 +351,84 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * 256;
       if (ti.kind == 0) {
         // projection tile: columns 0..r-1 = t, column r = gate logit
-        float lv[16];
-        tmem_ld16(taddr + (a.r / 16) * 16, lv);
-        const float g = sigmoidf_(lv[0] + a.b_g);
+        __nv_bfloat16* gdst = a.gt + (size_t)m * a.r;
+        float g;
+        if (a.gate_kind == 1) {
+          // rank gate (summary section 2.1 A): u = relu(W1 t + b1),
+          // gamma = sigmoid(W2 u + b2), gt = bf16(alpha gamma t); this
+          // thread's token row, t read from TMEM twice
+          float u[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) u[i] = i < a.gate_h ? __ldg(a.gb1 + i) : 0.f;
+          for (int c0 = 0; c0 < a.r; c0 += 16) {
+            float tv[16];
+            tmem_ld16(taddr + c0, tv);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < a.gate_h) {
+                const float4* w = reinterpret_cast<const float4*>(a.gw1 + (size_t)i * a.r + c0);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                  const float4 wv = __ldg(w + q4);
+                  u[i] = fmaf(wv.x, tv[4 * q4], u[i]);
+                  u[i] = fmaf(wv.y, tv[4 * q4 + 1], u[i]);
+                  u[i] = fmaf(wv.z, tv[4 * q4 + 2], u[i]);
+                  u[i] = fmaf(wv.w, tv[4 * q4 + 3], u[i]);
+                }
+              }
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) u[i] = fmaxf(u[i], 0.f);
+          float gsum = 0.f;
+          for (int c0 = 0; c0 < a.r; c0 += 16) {
+            float tv[16];
+            tmem_ld16(taddr + c0, tv);
+            float o[16];
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int j = c0 + jj;
+              float z = __ldg(a.gb2 + j);
+              const float4* w = reinterpret_cast<const float4*>(a.gw2 + (size_t)j * a.gate_h);
+#pragma unroll
+              for (int i4 = 0; i4 < 8; ++i4)
+                if (4 * i4 < a.gate_h) {
+                  const float4 wv = __ldg(w + i4);
+                  z = fmaf(wv.x, u[4 * i4], z);
+                  z = fmaf(wv.y, u[4 * i4 + 1], z);
+                  z = fmaf(wv.z, u[4 * i4 + 2], z);
+                  z = fmaf(wv.w, u[4 * i4 + 3], z);
+                }
+              const float gam = sigmoidf_(z);
+              gsum += gam;
+              o[jj] = a.alpha * gam * tv[jj];
+            }
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
+            uint4* d4 = reinterpret_cast<uint4*>(gdst + c0);
+            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+          g = gsum / (float)a.r;  // the reported gate: mean of gamma
+        } else {
+          float lv[16];
+          tmem_ld16(taddr + (a.r / 16) * 16, lv);
+          g = sigmoidf_(lv[0] + a.b_g);
+          for (int c0 = 0; c0 < a.r; c0 += 16) {
+            float tv[16];
+            tmem_ld16(taddr + c0, tv);
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(g * tv[2 * i], g * tv[2 * i + 1]);
+            uint4* d4 = reinterpret_cast<uint4*>(gdst + c0);
+            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
         const bool valid = m < a.M;
         if (valid && a.gate_out) a.gate_out[m] = g;
         const unsigned below = __ballot_sync(0xffffffffu, valid && g < a.tau);
         if (lane == 0 && a.mask_count && below) atomicAdd(&a.hdr->ec_done, __popc(below));
-        __nv_bfloat16* gdst = a.gt + (size_t)m * a.r;
-        for (int c0 = 0; c0 < a.r; c0 += 16) {
-          float tv[16];
-          tmem_ld16(taddr + c0, tv);
-          uint32_t pk[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(g * tv[2 * i], g * tv[2 * i + 1]);
-          uint4* d4 = reinterpret_cast<uint4*>(gdst + c0);
-          d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
         asm volatile("fence.proxy.async.global;" ::: "memory");
         __threadfence();
         tc_fence_before();
@@ -503,6 +566,13 @@ int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
   a.with_ec = with_ec && L.r > 0;
   a.NE = 16 * ((a.r + 1 + 15) / 16);
   a.ec_steps = (a.r + TC_BK - 1) / TC_BK;
+  a.gate_kind = a.with_ec ? L.gate_kind : 0;
+  a.gate_h = L.gate_h;
+  a.gw1 = L.gw1;
+  a.gb1 = L.gb1;
+  a.gw2 = L.gw2;
+  a.gb2 = L.gb2;
+  a.alpha = L.alpha;
   CUtensorMap maps[5];
   memset(maps, 0, sizeof(maps));
   bool ok = tmap_2d_bf16(&maps[0], x, L.K, M, TC_BK, TC_BM) && tmap_packed_box(&maps[1], L.w, L.K, L.N, 1, TC_BN / 16);

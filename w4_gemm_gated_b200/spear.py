@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import dataclasses
 from dataclasses import dataclass
 
 import torch
@@ -32,6 +33,8 @@ PATH_DECODE = 1
 PATH_FUSED = 2
 PATH_UNFUSED = 3
 PATH_SEMIFUSED = 4
+GATE_SCALAR = 0
+GATE_RANK_MLP = 1
 PATH_NAMES = {PATH_DECODE: "decode", PATH_FUSED: "fused", PATH_UNFUSED: "unfused", PATH_SEMIFUSED: "semifused"}
 
 _vp = ctypes.c_void_p
@@ -47,6 +50,9 @@ class LayerStruct(ctypes.Structure):
         ("K", _i), ("N", _i), ("group", _i), ("r", _i),
         ("w_packed", _vp), ("scales", _vp), ("AgT", _vp), ("BpT", _vp),
         ("b_g", _f), ("gate_tau", _f),
+        ("gate_kind", _i), ("gate_hidden", _i),
+        ("gate_w1", _vp), ("gate_b1", _vp), ("gate_w2", _vp), ("gate_b2", _vp),
+        ("gate_alpha", _f),
     ]
 
 
@@ -184,12 +190,37 @@ class Layer:
     BpT: torch.Tensor | None
     b_g: float
     gate_tau: float = 0.1
+    # the pages' per-rank gate gamma(t) = sigmoid(W2 relu(W1 t + b1) + b2) (fp32 device tensors)
+    gate_kind: int = GATE_SCALAR
+    gate_w1: torch.Tensor | None = None   # h x r
+    gate_b1: torch.Tensor | None = None   # h
+    gate_w2: torch.Tensor | None = None   # r x h
+    gate_b2: torch.Tensor | None = None   # r
+    gate_alpha: float = 1.0
 
     def struct(self) -> LayerStruct:
+        rank = self.gate_kind == GATE_RANK_MLP
         return LayerStruct(self.K, self.N, self.group, self.r, _ptr(self.w_packed), _ptr(self.scales),
                            _ptr(self.AgT) if self.AgT is not None else None,
                            _ptr(self.BpT) if self.BpT is not None else None,
-                           float(self.b_g), float(self.gate_tau))
+                           float(self.b_g), float(self.gate_tau),
+                           int(self.gate_kind), int(self.gate_w1.shape[0]) if rank else 0,
+                           _ptr(self.gate_w1) if rank else None, _ptr(self.gate_b1) if rank else None,
+                           _ptr(self.gate_w2) if rank else None, _ptr(self.gate_b2) if rank else None,
+                           float(self.gate_alpha))
+
+
+def with_rank_gate(layer: Layer, W1: torch.Tensor, b1: torch.Tensor, W2: torch.Tensor, b2: torch.Tensor,
+                   alpha: float) -> Layer:
+    """The same prepared layer with the pages' per-rank gate instead of the scalar one
+    (parameters copied to contiguous fp32 device tensors)."""
+    dev = layer.w_packed.device
+
+    def f32(t):
+        return t.detach().to(device=dev, dtype=torch.float32).contiguous()
+
+    return dataclasses.replace(layer, gate_kind=GATE_RANK_MLP, gate_w1=f32(W1), gate_b1=f32(b1),
+                               gate_w2=f32(W2), gate_b2=f32(b2), gate_alpha=float(alpha))
 
 
 def prepare_layer(W: torch.Tensor, group: int, A: torch.Tensor | None, B: torch.Tensor | None,
