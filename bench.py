@@ -355,12 +355,11 @@ def main():
     achieved = tot_bytes / (el_ms * 1e-3 / args.steps) / 1e9
 
     # per-M launch durations (informative): event-free graphs of one M only
-    mean_us = {}
-    for M in MS:
+    def per_launch_us(lays, M):
         gm = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gm, stream=stream):
             for i in range(3 * ncopy):
-                S.forward(layers[i % ncopy], xs[M], ws, y=ys[M], stream=stream)
+                S.forward(lays[i % ncopy], xs[M], ws, y=ys[M], stream=stream)
         with torch.cuda.stream(stream):
             gm.replay()
             m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -369,7 +368,17 @@ def main():
                 gm.replay()
             m1.record(stream)
         m1.synchronize()
-        mean_us[M] = m0.elapsed_time(m1) * 1e3 / (4 * 3 * ncopy)
+        return m0.elapsed_time(m1) * 1e3 / (4 * 3 * ncopy)
+
+    mean_us = {M: per_launch_us(layers, M) for M in MS}
+    # the pages' per-rank gate gamma(t) (bottleneck h = 16) on the same layers
+    rng = np.random.default_rng(7)
+    rg = [torch.from_numpy(v.astype(np.float32)).to(dev) for v in
+          (rng.standard_normal((16, R_)) / np.sqrt(R_), rng.standard_normal(16) * 0.1,
+           rng.standard_normal((R_, 16)) / 4.0, rng.standard_normal(R_) - 0.5)]
+    rank_layers = [S.with_rank_gate(lay, *rg, 1.0) for lay in layers]
+    rank_us = {M: per_launch_us(rank_layers, M) for M in (1, 16)}
+    assert S.read_status(ws, stream=stream) == S.OK
 
     tokens_per_step = sum(MS)
     value = whole_job_rate(tokens_per_step, args.steps, world, el_ms)
@@ -452,6 +461,9 @@ def main():
                      "peak_source": f"{peak_src} hbm_gbs"},
         "ec_overhead": {"m16_with_ec_us": mean_us[16], "m16_ec_disabled_us": noec_us,
                         "overhead": mean_us[16] / noec_us - 1.0},
+        "rank_gate": {"per_launch_us": rank_us, "hidden": 16,
+                      "vs_scalar_gate": {M: rank_us[M] / mean_us[M] - 1.0 for M in rank_us},
+                      "form": "y = xW + alpha (t * sigmoid(W2 relu(W1 t + b1) + b2)) B, t = xA"},
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(2 * M * K_ for M in MS), "d2h_bytes_per_step": sum(2 * M * N_ for M in MS),
                 "steps": e2e_steps, "api": "w4_gemm_gated_b200.spear.forward (eager, pinned host buffers)"},
@@ -688,13 +700,18 @@ def bench_prefill(S, synth, dev, stream, bf16, tc_peak):
         L = synth.prefill()
         lay = S.prepare_layer(torch.from_numpy(L.W).to(dev), 0, bf16(L.A), bf16(L.B), bf16(L.w_g), L.b_g)
         plain = S.Layer(4096, 4096, 0, 0, lay.w_packed, lay.scales, None, None, 0.0)
+        rng = np.random.default_rng(7)
+        rank = S.with_rank_gate(lay, *[torch.from_numpy(v.astype(np.float32)) for v in
+                                       (rng.standard_normal((16, 64)) / 8.0, rng.standard_normal(16) * 0.1,
+                                        rng.standard_normal((64, 16)) / 4.0, rng.standard_normal(64) - 0.5)], 1.0)
         x = bf16(L.x)
         y = torch.empty((2048, 4096), dtype=torch.bfloat16, device=dev)
         ws = S.make_workspace(lay, 2048)
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         res = {}
         for name, ly, path in (("fused", lay, S.PATH_FUSED), ("unfused", lay, S.PATH_UNFUSED),
-                               ("ec_disabled", plain, S.PATH_FUSED)):
+                               ("semifused", lay, S.PATH_SEMIFUSED), ("ec_disabled", plain, S.PATH_FUSED),
+                               ("fused_rank_gate", rank, S.PATH_FUSED)):
             ts = []
             with torch.cuda.stream(stream):
                 for i in range(13):
@@ -712,7 +729,8 @@ def bench_prefill(S, synth, dev, stream, bf16, tc_peak):
         fl = alg_flops(2048, 4096, 4096, 64)
         tf = fl / (res["fused"] * 1e-6) / 1e12
         return {"workload": "prefill GEMM M=2048 K=N=4096 r=64 (attention o-projection)",
-                "fused_us": res["fused"], "unfused_us": res["unfused"], "ec_disabled_us": res["ec_disabled"],
+                "fused_us": res["fused"], "unfused_us": res["unfused"], "semifused_us": res["semifused"],
+                "ec_disabled_us": res["ec_disabled"], "fused_rank_gate_us": res["fused_rank_gate"],
                 "tokens_per_s": 2048 / (res["fused"] * 1e-6), "tflops": tf,
                 "roofline": {"bound": "tensor", "achieved": tf, "peak": tc_peak, "unit": "TFLOP/s",
                              "frac": tf / tc_peak},

@@ -252,11 +252,11 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
   const int sms = sm_count();
   if (path == SPEAR_PATH_DECODE) {
     if (M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs M <= 16 (M=%d)", M);
-    if (!decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind))
+    if (!decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind, L.gate_h))
       return launch_decode2(L, x, M, y, hdr, tbuf, gate_out, mask_count, false, st);
     if (L.gate_kind)
       return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: the rank gate needs the main decode kernel (%s)",
-                       decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind));
+                       decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind, L.gate_h));
     DecodePlan p = plan_decode(M, L.K, L.N, L.r, L.group, sms);
     const char* why = check_decode_plan(p);
     if (why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", why);
@@ -269,7 +269,7 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
     L0.bpt = nullptr;
     L0.gate_kind = 0;
     int rc;
-    if (M <= 16 && !decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind)) {
+    if (M <= 16 && !decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind, L.gate_h)) {
       rc = launch_decode2(L0, x, M, y, hdr, tbuf, L.r > 0 ? nullptr : gate_out, L.r > 0 ? nullptr : mask_count,
                           false, st);
       if (rc || L.r == 0) return rc;
@@ -307,7 +307,7 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
     L0.agt = nullptr;
     L0.bpt = nullptr;
     L0.gate_kind = 0;
-    const bool d2 = M <= 16 && !decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind);
+    const bool d2 = M <= 16 && !decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind, L.gate_h);
     auto gemm = [&](float* go, int* mc) {
       if (d2) return launch_decode2(L0, x, M, y, hdr, tbuf, go, mc, false, st);
       TcPlan p = plan_tc(M, L.K, L.N, 0, L.group, sms);

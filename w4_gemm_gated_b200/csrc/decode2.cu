@@ -93,11 +93,13 @@ struct D2Args {
 
 // Shared-memory carve-up (same on host and device).
 struct D2Smem {
-  uint32_t ring, red, recv, park, bps, scs, ts, gts, gsc, stage, bars, total;
+  uint32_t ring, red, recv, park, bps, scs, ts, gts, gsc, gpar, stage, bars, total;
 };
+// rank-gate parameters staged in shared memory: W1 [h][r], W2 [r][h], b1 [h], b2 [r] (fp32)
+__host__ __device__ __forceinline__ uint32_t d2_gpar_floats(int h, int r) { return 2 * h * r + h + r; }
 __host__ __device__ __forceinline__ uint32_t d2_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 __host__ __device__ __forceinline__ D2Smem d2_smem(int MT, int nslot, int CS, int own_cap, int r, int ES,
-                                                   int gate_kind) {
+                                                   int gate_kind, int gate_h) {
   D2Smem s;
   const uint32_t NT = MT / 8;
   uint32_t off = 0;
@@ -119,6 +121,8 @@ __host__ __device__ __forceinline__ D2Smem d2_smem(int MT, int nslot, int CS, in
   off += d2_up(MT * (r + 8) * 2, 16);
   s.gsc = off;  // rank gate: hidden activations [MT][32] fp32
   off += gate_kind ? MT * 32 * 4 : 0;
+  s.gpar = off;  // rank gate: W1, W2, b1, b2
+  off += gate_kind ? d2_up(d2_gpar_floats(gate_h, r) * 4, 16) : 0;
   s.stage = off;
   off += MT * 32;
   s.bars = off;
@@ -337,7 +341,8 @@ __device__ __forceinline__ void d2_ts_fetch(const unsigned long long* tt, unsign
 // gt[m][j] = bf16(alpha gamma_j t[m][j]), and the reported gate is the mean of
 // gamma.  CTA 0 also writes the gate outputs and the mask count.
 template <int MT>
-__device__ void d2_build_gt(const D2Args& a, const unsigned long long* ts, __nv_bfloat16* gts, float* gsc, int lane) {
+__device__ void d2_build_gt(const D2Args& a, const unsigned long long* ts, __nv_bfloat16* gts, float* gsc,
+                            const float* gpar, int lane) {
   auto tval = [&](int m, int row) {
     return __uint_as_float((uint32_t)ts[((row >> 4) * MT + m) * 16 + (row & 15)]);
   };
@@ -345,15 +350,20 @@ __device__ void d2_build_gt(const D2Args& a, const unsigned long long* ts, __nv_
   float g;  // lane m: token m's gate
   if (a.gate_kind == 1) {
     const int h = a.gate_h, r = a.r;
+    const float* W1 = gpar;              // [h][r]
+    const float* W2 = gpar + h * r;      // [r][h]
+    const float* B1 = gpar + 2 * h * r;  // [h]
+    const float* B2 = B1 + h;            // [r]
     // hidden activations of the live tokens
     for (int idx = lane; idx < MT * h; idx += 32) {
       const int m = idx / h, i = idx - m * h;
       float v = 0.f;
       if (m < a.M) {
-        v = __ldg(a.gb1 + i);
-        const float4* w = reinterpret_cast<const float4*>(a.gw1 + (size_t)i * r);
+        v = B1[i];
+        const float4* w = reinterpret_cast<const float4*>(W1 + i * r);
+#pragma unroll 4
         for (int j4 = 0; j4 < r / 4; ++j4) {
-          const float4 wv = __ldg(w + j4);
+          const float4 wv = w[j4];
           v = fmaf(wv.x, tval(m, 4 * j4), v);
           v = fmaf(wv.y, tval(m, 4 * j4 + 1), v);
           v = fmaf(wv.z, tval(m, 4 * j4 + 2), v);
@@ -372,10 +382,12 @@ __device__ void d2_build_gt(const D2Args& a, const unsigned long long* ts, __nv_
       const int m = idx / r, j = idx - m * r;
       float gam = 0.f, o = 0.f;
       if (m < a.M) {
-        float z = __ldg(a.gb2 + j);
-        const float4* w = reinterpret_cast<const float4*>(a.gw2 + (size_t)j * h);
-        for (int i4 = 0; i4 < h / 4; ++i4) {
-          const float4 wv = __ldg(w + i4);
+        float z = B2[j];
+        const float4* w = reinterpret_cast<const float4*>(W2 + j * h);
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          if (4 * i4 >= h) break;
+          const float4 wv = w[i4];
           z = fmaf(wv.x, gsc[m * 32 + 4 * i4], z);
           z = fmaf(wv.y, gsc[m * 32 + 4 * i4 + 1], z);
           z = fmaf(wv.z, gsc[m * 32 + 4 * i4 + 2], z);
@@ -437,7 +449,7 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
   // 1024-byte aligned base, derived from the shared array itself so that the
   // compiler keeps every access in the shared window (ld/st.shared)
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const D2Smem SL = d2_smem(MT, a.nslot, a.CS, a.own_cap, a.r, a.ES, a.gate_kind);
+  const D2Smem SL = d2_smem(MT, a.nslot, a.CS, a.own_cap, a.r, a.ES, a.gate_kind, a.gate_h);
   uint8_t* ring = sm + SL.ring;
   float4* red = reinterpret_cast<float4*>(sm + SL.red);
   float4* recv = reinterpret_cast<float4*>(sm + SL.recv);
@@ -447,6 +459,7 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
   unsigned long long* ts = reinterpret_cast<unsigned long long*>(sm + SL.ts);
   __nv_bfloat16* gts = reinterpret_cast<__nv_bfloat16*>(sm + SL.gts);
   float* gsc = reinterpret_cast<float*>(sm + SL.gsc);
+  float* gpar = reinterpret_cast<float*>(sm + SL.gpar);
   __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sm + SL.stage);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + SL.bars);
   uint64_t* empty = full + a.nslot;
@@ -751,6 +764,20 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
     // within the cluster (rank order), publishes EC strips, fetches the whole EC
     // projection without blocking, and runs (or parks) the strip epilogues.
     const int rho = lane >> 2, c = lane & 3;
+    if (a.gate_kind == 1) {
+      // rank-gate parameters into shared memory while the first partials are
+      // computed (all four arrays have a multiple of 4 floats, 16-byte aligned)
+      const int h = a.gate_h, r = a.r;
+      auto stage4 = [&](const float* src, float* dst, int n) {
+        for (int i = lane; i < n / 4; i += 32)
+          reinterpret_cast<float4*>(dst)[i] = __ldg(reinterpret_cast<const float4*>(src) + i);
+      };
+      stage4(a.gw1, gpar, h * r);
+      stage4(a.gw2, gpar + h * r, r * h);
+      stage4(a.gb1, gpar + 2 * h * r, h);
+      stage4(a.gb2, gpar + 2 * h * r + h, r);
+      __syncwarp();
+    }
     if (a.CS > 1) asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
     const uint32_t tag = (uint32_t)(*reinterpret_cast<volatile int*>(&a.hdr->d2_epoch)) + 1u;
     // EC projection state: 0 idle, 1 probe in flight, 2 full fetch in flight, 3 gate and gt ready.
@@ -775,7 +802,7 @@ __global__ void __launch_bounds__(D2_THREADS, 2)
         }
         tok = __all_sync(FULL, tok);
         if (tok && gst == 2) {
-          d2_build_gt<MT>(a, ts, gts, gsc, lane);
+          d2_build_gt<MT>(a, ts, gts, gsc, gpar, lane);
           gst = 3;
           // every CTA reads the projection once; the last reader advances the epoch
           if (lane == 0) obs_prev = atomicAdd(&a.hdr->gt_obs, 1);
@@ -1037,7 +1064,7 @@ static cudaError_t d2_attrs(size_t smem) {
   return cudaSuccess;
 }
 
-static D2Plan make_d2_plan(int MT, int K, int N, int r, int sms, int gate_kind) {
+static D2Plan make_d2_plan(int MT, int K, int N, int r, int sms, int gate_kind, int gate_h) {
   D2Plan p = {};
   p.MT = MT;
   p.why = nullptr;
@@ -1094,26 +1121,26 @@ static D2Plan make_d2_plan(int MT, int K, int N, int r, int sms, int gate_kind) 
     p.why = "too many strips per CTA for the decode kernel";
     return p;
   }
-  const D2Smem s0 = d2_smem(MT, 0, p.CS, own, r, p.ES, gate_kind);
+  const D2Smem s0 = d2_smem(MT, 0, p.CS, own, r, p.ES, gate_kind, gate_h);
   const size_t per_slot = D2_SLOT + 16;
   p.nslot = (int)std::min<size_t>(D2_MAXSLOT, (D2_SMEM_CAP - std::min<size_t>(s0.total, D2_SMEM_CAP)) / per_slot);
   if (p.nslot < 3) {
     p.why = "shared memory too small for the decode kernel's ring";
     return p;
   }
-  p.smem = d2_smem(MT, p.nslot, p.CS, own, r, p.ES, gate_kind).total;
+  p.smem = d2_smem(MT, p.nslot, p.CS, own, r, p.ES, gate_kind, gate_h).total;
   return p;
 }
 
-static const D2Plan& d2_plan(int MT, int K, int N, int r, int sms, int gate_kind) {
+static const D2Plan& d2_plan(int MT, int K, int N, int r, int sms, int gate_kind, int gate_h) {
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int, int, int, int, int>, D2Plan> cache;
+  static std::map<std::tuple<int, int, int, int, int, int, int, int>, D2Plan> cache;
   int dev = 0;
   cudaGetDevice(&dev);
-  const auto key = std::make_tuple(dev, MT, K, N, r, sms, gate_kind);
+  const auto key = std::make_tuple(dev, MT, K, N, r, sms, gate_kind, gate_kind ? gate_h : 0);
   std::lock_guard<std::mutex> lk(mu);
   auto it = cache.find(key);
-  if (it == cache.end()) it = cache.emplace(key, make_d2_plan(MT, K, N, r, sms, gate_kind)).first;
+  if (it == cache.end()) it = cache.emplace(key, make_d2_plan(MT, K, N, r, sms, gate_kind, gate_h)).first;
   return it->second;
 }
 
@@ -1122,9 +1149,9 @@ size_t decode2_tt_bytes(int r) {
   return (size_t)ES * 16 * 16 * 8;
 }
 
-const char* decode2_unsupported(int M, int K, int N, int r, int gate_kind) {
+const char* decode2_unsupported(int M, int K, int N, int r, int gate_kind, int gate_h) {
   if (M < 1 || M > 16) return "the decode kernel needs 1 <= M <= 16";
-  return d2_plan(M <= 8 ? 8 : 16, K, N, r, device_sm_count(), gate_kind).why;
+  return d2_plan(M <= 8 ? 8 : 16, K, N, r, device_sm_count(), gate_kind, gate_h).why;
 }
 
 template <int MT, int KTW, bool GROUP>
@@ -1182,7 +1209,7 @@ int launch_decode2(const LayerView& Lv, const __nv_bfloat16* x, int M, __nv_bflo
   if (M < 1 || M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs 1 <= M <= 16 (M=%d)", M);
   const int MT = M <= 8 ? 8 : 16;
   const int gk = Lv.r > 0 ? Lv.gate_kind : 0;
-  const D2Plan& p = d2_plan(MT, Lv.K, Lv.N, Lv.r, device_sm_count(), gk);
+  const D2Plan& p = d2_plan(MT, Lv.K, Lv.N, Lv.r, device_sm_count(), gk, Lv.gate_h);
   if (p.why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", p.why);
   if (ec_only && Lv.r == 0) return set_error(SPEAR_ERR_INVALID_ARG, "EC-only launch without an EC");
   D2Args a = {};

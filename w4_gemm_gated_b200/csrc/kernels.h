@@ -56,7 +56,7 @@ int launch_decode(const DecodePlan& p, const LayerView& L, const __nv_bfloat16* 
 
 // ---- decode path for back-to-back launches (decode2.cu) ----
 // null if the kernel can run (M, K, N, r), else the reason
-const char* decode2_unsupported(int M, int K, int N, int r, int gate_kind);
+const char* decode2_unsupported(int M, int K, int N, int r, int gate_kind, int gate_h);
 // bytes of tagged EC projection words the kernel needs in the workspace
 size_t decode2_tt_bytes(int r);
 int launch_decode2(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, WsHeader* hdr, void* tt,

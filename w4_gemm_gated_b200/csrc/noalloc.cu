@@ -73,7 +73,7 @@ extern "C" int spear_linear_forward_decode_noalloc(const spear_layer* layer, con
       (gate_out && (reinterpret_cast<uintptr_t>(gate_out) & 3)) ||
       (mask_count && (reinterpret_cast<uintptr_t>(mask_count) & 3)))
     return set_error(SPEAR_ERR_ALIGNMENT, "x and y must be 16-byte aligned");
-  const bool v2 = decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind) == nullptr;
+  const bool v2 = decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind, L.gate_h) == nullptr;
   if (!v2 && L.gate_kind)
     return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: the rank gate needs the main decode kernel");
   if (v2 && decode2_tt_bytes(L.r) > kNoAllocEcp)

@@ -48,6 +48,9 @@ constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;      // 32 KB
 constexpr int TC_P_BYTES = TC_BN * TC_BK / 2;      // 8 KB
 constexpr int TC_STAGE_BYTES = TC_X_BYTES + TC_B_BYTES + TC_P_BYTES;
 constexpr int TC_SMEM = TC_STAGES * TC_STAGE_BYTES + 1024 /* barriers */ + 1024 /* alignment */;
+// rank-gate parameters (W1 [h][r], W2 [r][h], b1 [h], b2 [r], fp32) after the barriers
+__host__ __device__ constexpr int tc_gpar_bytes(int h, int r) { return (2 * h * r + h + r) * 4; }
+constexpr int TC_SMEM_MAX = TC_SMEM + tc_gpar_bytes(32, 128);
 
 struct TcArgs {
   const __half* scales;
@@ -209,6 +212,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t* acc_empty = acc_full + 2;        // [2]
   uint32_t* tmem_base_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_holder + 1);
+  float* gpar = reinterpret_cast<float*>(ps + TC_STAGES * TC_P_BYTES + 1024);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int epoch = *reinterpret_cast<volatile int*>(&a.hdr->epoch);
@@ -338,6 +342,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   } else if (warp < 6) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter of this warp
+    if (a.gate_kind == 1) {
+      // rank-gate parameters into shared memory (the 4 epilogue warps; every
+      // array has a multiple of 4 floats and is 16-byte aligned)
+      const int h = a.gate_h, r = a.r, et = threadIdx.x - 64;
+      auto stage4 = [&](const float* src, float* dst, int n) {
+        for (int i = et; i < n / 4; i += 128)
+          reinterpret_cast<float4*>(dst)[i] = __ldg(reinterpret_cast<const float4*>(src) + i);
+      };
+      stage4(a.gw1, gpar, h * r);
+      stage4(a.gw2, gpar + h * r, r * h);
+      stage4(a.gb1, gpar + 2 * h * r, h);
+      stage4(a.gb2, gpar + 2 * h * r + h, r);
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+    }
+    const float* W1 = gpar;
+    const float* W2 = gpar + a.gate_h * a.r;
+    const float* B1 = gpar + 2 * a.gate_h * a.r;
+    const float* B2 = B1 + a.gate_h;
     int buf = 0;
     uint32_t aph[2] = {0, 0};
     bool ok = true;
@@ -359,17 +381,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           // thread's token row, t read from TMEM twice
           float u[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = i < a.gate_h ? __ldg(a.gb1 + i) : 0.f;
+          for (int i = 0; i < 32; ++i) u[i] = i < a.gate_h ? B1[i] : 0.f;
           for (int c0 = 0; c0 < a.r; c0 += 16) {
             float tv[16];
             tmem_ld16(taddr + c0, tv);
 #pragma unroll
             for (int i = 0; i < 32; ++i)
               if (i < a.gate_h) {
-                const float4* w = reinterpret_cast<const float4*>(a.gw1 + (size_t)i * a.r + c0);
+                const float4* w = reinterpret_cast<const float4*>(W1 + i * a.r + c0);
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
-                  const float4 wv = __ldg(w + q4);
+                  const float4 wv = w[q4];
                   u[i] = fmaf(wv.x, tv[4 * q4], u[i]);
                   u[i] = fmaf(wv.y, tv[4 * q4 + 1], u[i]);
                   u[i] = fmaf(wv.z, tv[4 * q4 + 2], u[i]);
@@ -387,12 +409,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
               const int j = c0 + jj;
-              float z = __ldg(a.gb2 + j);
-              const float4* w = reinterpret_cast<const float4*>(a.gw2 + (size_t)j * a.gate_h);
+              float z = B2[j];
+              const float4* w = reinterpret_cast<const float4*>(W2 + j * a.gate_h);
 #pragma unroll
               for (int i4 = 0; i4 < 8; ++i4)
                 if (4 * i4 < a.gate_h) {
-                  const float4 wv = __ldg(w + i4);
+                  const float4 wv = w[i4];
                   z = fmaf(wv.x, u[4 * i4], z);
                   z = fmaf(wv.y, u[4 * i4 + 1], z);
                   z = fmaf(wv.z, u[4 * i4 + 2], z);
@@ -533,12 +555,13 @@ static int launch_tc_t(const TcPlan& p, const TcArgs& a, const CUtensorMap* maps
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(tc_kernel<GROUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+    attr_err = cudaFuncSetAttribute(tc_kernel<GROUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM_MAX);
   });
   if (attr_err != cudaSuccess) return set_cuda_error("cudaFuncSetAttribute(tc)", attr_err);
   const int ntiles = (a.with_ec ? a.Mb : 0) + a.Mb * a.Nb;
   const int grid = ntiles < p.grid ? ntiles : p.grid;
-  tc_kernel<GROUP><<<grid, TC_THREADS, p.smem, st>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4]);
+  const size_t smem = p.smem + (a.gate_kind == 1 ? tc_gpar_bytes(a.gate_h, a.r) : 0);
+  tc_kernel<GROUP><<<grid, TC_THREADS, smem, st>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4]);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPEAR_OK : set_cuda_error("tc kernel launch", e);
 }
