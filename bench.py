@@ -513,7 +513,7 @@ def run_sweep(args):
         return float(np.median(ts))
 
     names = S.PATH_NAMES
-    points, good = [], 0
+    points, good, failures = [], 0, []
     S.dispatch_clear()
     t_start = time.perf_counter()
     for K, N in SWEEP_KN:
@@ -527,10 +527,19 @@ def run_sweep(args):
                 ws = S.make_workspace(layer, max(SWEEP_MS))
                 y_all = torch.empty((max(SWEEP_MS), N), dtype=torch.bfloat16, device="cuda")
                 S.dispatch_tune(layer, list(SWEEP_MS), x_all, y_all, ws, flush=flush, reps=10)
+                st = S.read_status(ws)
+                if st != S.OK:
+                    failures.append({"K": K, "N": N, "r": r, "group": group, "stage": "tune", "status": st})
                 for M in SWEEP_MS:
                     paths = [S.PATH_FUSED, S.PATH_UNFUSED, S.PATH_SEMIFUSED] + ([S.PATH_DECODE] if M <= 16 else [])
                     x = x_all[:M].contiguous()
-                    t = {p: median_us(layer, x, y_all[:M], ws, p, 10) for p in paths}
+                    t = {}
+                    for p in paths:
+                        t[p] = median_us(layer, x, y_all[:M], ws, p, 10)
+                        st = S.read_status(ws)
+                        if st != S.OK:
+                            failures.append({"K": K, "N": N, "r": r, "group": group, "M": M, "path": names[p],
+                                             "status": st})
                     choice = S.dispatch_choice(layer, M)
                     best = min(t.values())
                     ok = t[choice] <= max(1.05 * best, best + 2.0)
@@ -540,15 +549,16 @@ def run_sweep(args):
                                    "us": {names[p]: round(v, 2) for p, v in t.items()},
                                    "choice": names[choice], "choice_ok": bool(ok),
                                    "tflops_best": round(fl / (best * 1e-6) / 1e12, 2)})
-                if S.read_status(ws) != S.OK:
-                    raise SystemExit("device status not OK during the sweep")
                 del layer, ws, y_all
         del W, x_all
     S.dispatch_clear()
     print(json.dumps({"sweep": "dispatch (M x (K,N) x r x scale kind)", "points": len(points),
                       "dispatcher_within_5pct": good, "seconds": round(time.perf_counter() - t_start, 1),
+                      "device_status_failures": failures,
                       "timing": "median of 10 launches, L2 flushed (256 MB write) before each",
                       "table": points}))
+    if failures:
+        sys.exit(1)
 
 
 STACK_SHAPES = ((4096, 4096), (4096, 4096), (4096, 4096), (4096, 4096),  # q, k, v, o

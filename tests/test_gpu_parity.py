@@ -266,3 +266,17 @@ def test_workspace_reuse_across_paths_and_sizes(S):
         torch.cuda.synchronize()
         assert_close(y, O.linear(x, q, s, 0, L.A, L.B, L.w_g, L.b_g)[0])
     assert S.read_status(ws) == S.OK
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_decode_long_k_rank128_clusters_resident(S, M):
+    """K = 14336 splits K over clusters of 7 CTAs; with r = 128 the 9 EC strips
+    sit in clusters across the grid.  Every cluster must be resident at once
+    (each CTA waits for every EC strip), so the plan caps the cluster count at
+    what the device holds: the call finishes with status OK and matches."""
+    L = synth.make_layer(M, 14336, 4096, 128, b_g=-1.0, x_kind="t3", seed=77 + M)
+    layer = prepared(S, L, 0)
+    y, g, _, _ = run(S, layer, L.x, S.PATH_DECODE, gate=True)
+    y_ref, g_ref, _, _ = oracle_ref(L, 0)
+    assert_close(y, y_ref)
+    assert np.max(np.abs(g.cpu().numpy() - g_ref)) <= GATE_TOL

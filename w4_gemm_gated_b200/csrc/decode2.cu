@@ -1064,7 +1064,7 @@ static cudaError_t d2_attrs(size_t smem) {
   return cudaSuccess;
 }
 
-static D2Plan make_d2_plan(int MT, int K, int N, int r, int sms, int gate_kind, int gate_h) {
+static D2Plan make_d2_plan(int MT, int K, int N, int r, int sms, int gate_kind, int gate_h, int nc_cap) {
   D2Plan p = {};
   p.MT = MT;
   p.why = nullptr;
@@ -1091,8 +1091,10 @@ static D2Plan make_d2_plan(int MT, int K, int N, int r, int sms, int gate_kind, 
   p.ES = r > 0 ? (r + 1 + 15) / 16 : 0;
   const int NS = N / 16;
   // two CTAs per SM per launch: the next launch takes an SM's halves as this
-  // one leaves them (measured faster than one CTA per SM beside the next launch)
-  int NC = std::max(1, 2 * sms / p.CS);
+  // one leaves them (measured faster than one CTA per SM beside the next
+  // launch); never more clusters than can be resident at once (nc_cap), since
+  // every CTA waits for the EC strips of other clusters
+  int NC = std::max(1, std::min(2 * sms / p.CS, nc_cap));
   NC = std::min(NC, std::max(1, NS + p.ES));
   NC = std::min(NC, D2_MAXCL);
   p.NC = NC;
@@ -1132,16 +1134,89 @@ static D2Plan make_d2_plan(int MT, int K, int N, int r, int sms, int gate_kind, 
   return p;
 }
 
+// Clusters of this kernel instance that fit on the device at once (cluster
+// size CS, `smem` bytes each); 0 if the query fails.
+template <int MT, int KTW>
+static int d2_max_clusters_t(int CS, size_t smem) {
+  if (d2_attrs<MT, KTW, false>(smem) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  int n = 0;
+  if (CS == 1) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode2_kernel<MT, KTW, false>, D2_THREADS, smem) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    return per_sm * device_sm_count();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CS);
+  cfg.blockDim = dim3(D2_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+  attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicySpread;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (cudaOccupancyMaxActiveClusters(&n, decode2_kernel<MT, KTW, false>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+static int d2_max_clusters(int MT, int KTW, int CS, size_t smem) {
+  if (MT == 8) {
+    switch (KTW) {
+      case 8: return d2_max_clusters_t<8, 8>(CS, smem);
+      case 4: return d2_max_clusters_t<8, 4>(CS, smem);
+      case 2: return d2_max_clusters_t<8, 2>(CS, smem);
+      default: return d2_max_clusters_t<8, 1>(CS, smem);
+    }
+  }
+  switch (KTW) {
+    case 8: return d2_max_clusters_t<16, 8>(CS, smem);
+    case 4: return d2_max_clusters_t<16, 4>(CS, smem);
+    case 2: return d2_max_clusters_t<16, 2>(CS, smem);
+    default: return d2_max_clusters_t<16, 1>(CS, smem);
+  }
+}
+
+// The plan for a shape, with its clusters capped at what is resident at once.
 static const D2Plan& d2_plan(int MT, int K, int N, int r, int sms, int gate_kind, int gate_h) {
   static std::mutex mu;
   static std::map<std::tuple<int, int, int, int, int, int, int, int>, D2Plan> cache;
   int dev = 0;
   cudaGetDevice(&dev);
-  const auto key = std::make_tuple(dev, MT, K, N, r, sms, gate_kind, gate_kind ? gate_h : 0);
+  const int gh = gate_kind ? gate_h : 0;
+  const auto key = std::make_tuple(dev, MT, K, N, r, sms, gate_kind, gh);
   std::lock_guard<std::mutex> lk(mu);
   auto it = cache.find(key);
-  if (it == cache.end()) it = cache.emplace(key, make_d2_plan(MT, K, N, r, sms, gate_kind, gate_h)).first;
-  return it->second;
+  if (it != cache.end()) return it->second;
+  D2Plan p = make_d2_plan(MT, K, N, r, sms, gate_kind, gh, 1 << 30);
+  // fewer clusters give each more strips (more shared memory), which does not
+  // change residency while a CTA stays within the two-per-SM cap; re-check anyway
+  for (int iter = 0; !p.why; ++iter) {
+    const int mc = d2_max_clusters(MT, p.KTW, p.CS, p.smem);
+    if (mc <= 0) {
+      p.why = "cluster occupancy query failed for the decode kernel";
+    } else if (p.NC > mc) {
+      if (iter == 3)
+        p.why = "the decode kernel's clusters do not fit on the device at once";
+      else
+        p = make_d2_plan(MT, K, N, r, sms, gate_kind, gh, mc);
+    } else {
+      break;
+    }
+  }
+  return cache.emplace(key, std::move(p)).first->second;
 }
 
 size_t decode2_tt_bytes(int r) {
