@@ -40,17 +40,24 @@ namespace spear {
 constexpr int TC_BM = 128;
 constexpr int TC_BN = 256;
 constexpr int TC_BK = 64;
-constexpr int TC_STAGES = 3;
+// Ring stages: 4 fill the 227 KB of shared memory (one stage is reused every
+// TMA + dequant + MMA round trip, so more stages in flight run more steps per
+// round trip); 3 when the rank gate's parameters need shared memory too.
+constexpr int TC_STAGES = 4;
 constexpr int TC_PREFETCH = 8;  // k-steps of L2 prefetch ahead of the TMA loads
 constexpr int TC_THREADS = 14 * 32;  // producer, mma, 4 epilogue, 8 dequant warps
 constexpr int TC_X_BYTES = TC_BM * TC_BK * 2;      // 16 KB
 constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;      // 32 KB
 constexpr int TC_P_BYTES = TC_BN * TC_BK / 2;      // 8 KB
 constexpr int TC_STAGE_BYTES = TC_X_BYTES + TC_B_BYTES + TC_P_BYTES;
-constexpr int TC_SMEM = TC_STAGES * TC_STAGE_BYTES + 1024 /* barriers */ + 1024 /* alignment */;
+__host__ __device__ constexpr int tc_smem(int nst) { return nst * TC_STAGE_BYTES + 1024 /* barriers */ + 1024 /* alignment */; }
+constexpr int TC_SMEM = tc_smem(TC_STAGES);
 // rank-gate parameters (W1 [h][r], W2 [r][h], b1 [h], b2 [r], fp32) after the barriers
 __host__ __device__ constexpr int tc_gpar_bytes(int h, int r) { return (2 * h * r + h + r) * 4; }
-constexpr int TC_SMEM_MAX = TC_SMEM + tc_gpar_bytes(32, 128);
+constexpr int TC_SMEM_MAX = TC_SMEM > tc_smem(TC_STAGES - 1) + tc_gpar_bytes(32, 128)
+                                ? TC_SMEM
+                                : tc_smem(TC_STAGES - 1) + tc_gpar_bytes(32, 128);
+static_assert(TC_SMEM_MAX <= 227 * 1024, "tensor-core kernel shared memory");
 
 struct TcArgs {
   const __half* scales;
@@ -69,6 +76,7 @@ struct TcArgs {
   int gate_kind, gate_h;  // 0: scalar gate; 1: per-rank gamma(t) with bottleneck h
   const float *gw1, *gb1, *gw2, *gb2;
   float alpha;
+  int nst;                // ring stages (TC_STAGES, or one fewer with the rank gate)
 };
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -202,24 +210,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   // compiler keeps every access in the shared window (ld/st.shared)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* xs = smem;                                        // [STAGES][16 KB]
-  uint8_t* bs = smem + TC_STAGES * TC_X_BYTES;               // [STAGES][32 KB]
-  uint8_t* ps = bs + TC_STAGES * TC_B_BYTES;                 // [STAGES][8 KB]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + TC_STAGES * TC_P_BYTES);
+  const int NST = a.nst;
+  uint8_t* bs = smem + NST * TC_X_BYTES;                     // [NST][32 KB]
+  uint8_t* ps = bs + NST * TC_B_BYTES;                       // [NST][8 KB]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + NST * TC_P_BYTES);
   uint64_t* full = bars;                     // TMA loads of a stage landed
-  uint64_t* ready = bars + TC_STAGES;        // B operand of a stage ready (dequant warps)
-  uint64_t* empty = bars + 2 * TC_STAGES;    // MMAs of a stage done
-  uint64_t* acc_full = bars + 3 * TC_STAGES; // [2]
+  uint64_t* ready = bars + NST;              // B operand of a stage ready (dequant warps)
+  uint64_t* empty = bars + 2 * NST;          // MMAs of a stage done
+  uint64_t* acc_full = bars + 3 * NST;       // [2]
   uint64_t* acc_empty = acc_full + 2;        // [2]
   uint32_t* tmem_base_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_holder + 1);
-  float* gpar = reinterpret_cast<float*>(ps + TC_STAGES * TC_P_BYTES + 1024);
+  float* gpar = reinterpret_cast<float*>(ps + NST * TC_P_BYTES + 1024);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int epoch = *reinterpret_cast<volatile int*>(&a.hdr->epoch);
   const int ntiles = (a.with_ec ? a.Mb : 0) + a.Mb * a.Nb;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < TC_STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&ready[s], 8);
       mbar_init(&empty[s], 1);
@@ -296,7 +305,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tma_load_2d(smem_u32(xd), &tm_gt, &full[s], e * TC_BK, ti.mb * TC_BM);
             tma_load_2d(smem_u32(bd), &tm_bpt, &full[s], e * TC_BK, ti.nb * TC_BN);
           }
-          if (++s == TC_STAGES) {
+          if (++s == NST) {
             s = 0;
             ph ^= 1;
           }
@@ -328,7 +337,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           for (int kk = 0; kk < TC_BK / 16; ++kk)
             umma(d, ad + 2 * kk, bd + 2 * kk, idesc, (k > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&empty[s]);
-          if (++s == TC_STAGES) {
+          if (++s == NST) {
             s = 0;
             ph ^= 1;
           }
@@ -508,7 +517,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&ready[s]);
-        if (++s == TC_STAGES) {
+        if (++s == NST) {
           s = 0;
           ph ^= 1;
         }
@@ -560,7 +569,7 @@ static int launch_tc_t(const TcPlan& p, const TcArgs& a, const CUtensorMap* maps
   if (attr_err != cudaSuccess) return set_cuda_error("cudaFuncSetAttribute(tc)", attr_err);
   const int ntiles = (a.with_ec ? a.Mb : 0) + a.Mb * a.Nb;
   const int grid = ntiles < p.grid ? ntiles : p.grid;
-  const size_t smem = p.smem + (a.gate_kind == 1 ? tc_gpar_bytes(a.gate_h, a.r) : 0);
+  const size_t smem = a.gate_kind == 1 ? tc_smem(a.nst) + tc_gpar_bytes(a.gate_h, a.r) : tc_smem(a.nst);
   tc_kernel<GROUP><<<grid, TC_THREADS, smem, st>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4]);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPEAR_OK : set_cuda_error("tc kernel launch", e);
@@ -596,6 +605,7 @@ int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
   a.gw2 = L.gw2;
   a.gb2 = L.gb2;
   a.alpha = L.alpha;
+  a.nst = a.gate_kind == 1 ? TC_STAGES - 1 : TC_STAGES;
   CUtensorMap maps[5];
   memset(maps, 0, sizeof(maps));
   bool ok = tmap_2d_bf16(&maps[0], x, L.K, M, TC_BK, TC_BM) && tmap_packed_box(&maps[1], L.w, L.K, L.N, 1, TC_BN / 16);
