@@ -281,6 +281,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             if (k + TC_PREFETCH < KT) {
               tma_prefetch_2d(&tm_x, (k + TC_PREFETCH) * TC_BK, ti.mb * TC_BM);
               tma_prefetch_3d(&tm_w, 0, k + TC_PREFETCH, ti.nb * (TC_BN / 16));
+            } else {
+              // the tile's tail: warm its EC operands (L2 is coherent, so gt may
+              // be warmed before the projection is published) and the first
+              // k-steps of this CTA's next tile
+              const int j = k + TC_PREFETCH - KT;
+              if (j == 0 && a.with_ec)
+                for (int e = 0; e < a.ec_steps; ++e) {
+                  tma_prefetch_2d(&tm_bpt, e * TC_BK, ti.nb * TC_BN);
+                  tma_prefetch_2d(&tm_gt, e * TC_BK, ti.mb * TC_BM);
+                }
+              const int nt = tile + (int)gridDim.x;
+              if (nt < ntiles) {
+                const TileInfo tn = tile_info(a, nt);
+                if (tn.kind == 1 && j < KT) {
+                  tma_prefetch_2d(&tm_x, j * TC_BK, tn.mb * TC_BM);
+                  tma_prefetch_3d(&tm_w, 0, j, tn.nb * (TC_BN / 16));
+                }
+              }
             }
             if (k == 0)
               for (int pk = 1; pk < TC_PREFETCH && pk < KT; ++pk) {
