@@ -143,3 +143,16 @@ def test_one_workspace_across_paths_and_sizes(S):
         torch.cuda.synchronize()
         assert S.read_status(ws) == S.OK, (M, path)
         assert_close(y, O.linear(x, q, s, 0, L.A, L.B, L.w_g, L.b_g)[0])
+
+
+@pytest.mark.parametrize("M,group,r", [(512, 0, 64), (600, 128, 32), (1000, 0, 128), (1300, 128, 16)])
+def test_tall_tiles_ragged(S, M, group, r):
+    """From M = 512 the kernel uses 256-token tiles (two accumulators); ragged
+    M leaves a partial last block."""
+    L = synth.make_layer(M, 2048, 1024, r, b_g=-0.3, x_kind="t3", seed=700 + M)
+    layer = prepared(S, L, group)
+    y_ref, g_ref, _, _ = oracle_ref(L, group)
+    for path in (S.PATH_FUSED, S.PATH_UNFUSED):
+        y, g, cnt, _ = run(S, layer, L.x, path, gate=True)
+        assert_close(y, y_ref)
+        assert np.max(np.abs(g.cpu().numpy() - g_ref)) <= GATE_TOL

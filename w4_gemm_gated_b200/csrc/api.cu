@@ -129,7 +129,7 @@ static constexpr int kFlagCap = kMaxM / 16 + 64;  // 16-token blocks (+ slack)
 
 static WsLayout ws_layout_uncached(const LayerView& L, int M_max) {
   WsLayout w = {};
-  const int Mpad = ((M_max + 127) / 128) * 128;
+  const int Mpad = ((M_max + 255) / 256) * 256;  // tensor-core tiles of up to 256 tokens
   const int RT = 32 * ((128 / 16 + 2) / 2) + 16;  // row stride for the largest rank
   w.n_flags = kFlagCap;
   size_t off = kWsHeaderBytes;

@@ -37,26 +37,31 @@
 
 namespace spear {
 
-constexpr int TC_BM = 128;
+constexpr int TC_BM = 128;  // rows of one MMA (and of one TMEM accumulator)
 constexpr int TC_BN = 256;
 constexpr int TC_BK = 64;
-// Ring stages: 4 fill the 227 KB of shared memory (one stage is reused every
-// TMA + dequant + MMA round trip, so more stages in flight run more steps per
-// round trip); 3 when the rank gate's parameters need shared memory too.
+// Tiles are BMT = 128 or 256 tokens (template): a 256-token tile runs two
+// M = 128 MMAs per k-step into two accumulators, so each dequantised weight
+// tile and each ring round trip feed twice the tensor-core work.
+// Ring stages: as many as fit the 227 KB of shared memory (one stage is reused
+// every TMA + dequant + MMA round trip): 4 at BMT = 128 (3 with the rank gate's
+// parameters), 3 at BMT = 256.
 constexpr int TC_STAGES = 4;
 constexpr int TC_PREFETCH = 8;  // k-steps of L2 prefetch ahead of the TMA loads
 constexpr int TC_THREADS = 14 * 32;  // producer, mma, 4 epilogue, 8 dequant warps
-constexpr int TC_X_BYTES = TC_BM * TC_BK * 2;      // 16 KB
+constexpr int TC_X_BYTES = TC_BM * TC_BK * 2;      // 16 KB: x rows of one MMA
 constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;      // 32 KB
 constexpr int TC_P_BYTES = TC_BN * TC_BK / 2;      // 8 KB
-constexpr int TC_STAGE_BYTES = TC_X_BYTES + TC_B_BYTES + TC_P_BYTES;
-__host__ __device__ constexpr int tc_smem(int nst) { return nst * TC_STAGE_BYTES + 1024 /* barriers */ + 1024 /* alignment */; }
-constexpr int TC_SMEM = tc_smem(TC_STAGES);
+__host__ __device__ constexpr int tc_stage_bytes(int bmt) { return bmt * TC_BK * 2 + TC_B_BYTES + TC_P_BYTES; }
+__host__ __device__ constexpr int tc_smem(int nst, int bmt) {
+  return nst * tc_stage_bytes(bmt) + 1024 /* barriers */ + 1024 /* alignment */;
+}
+constexpr int TC_SMEM = tc_smem(TC_STAGES, 128);
 // rank-gate parameters (W1 [h][r], W2 [r][h], b1 [h], b2 [r], fp32) after the barriers
 __host__ __device__ constexpr int tc_gpar_bytes(int h, int r) { return (2 * h * r + h + r) * 4; }
-constexpr int TC_SMEM_MAX = TC_SMEM > tc_smem(TC_STAGES - 1) + tc_gpar_bytes(32, 128)
-                                ? TC_SMEM
-                                : tc_smem(TC_STAGES - 1) + tc_gpar_bytes(32, 128);
+constexpr int tc_max3(int a, int b, int c) { return a > b ? (a > c ? a : c) : (b > c ? b : c); }
+constexpr int TC_SMEM_MAX =
+    tc_max3(TC_SMEM, tc_smem(TC_STAGES - 1, 128) + tc_gpar_bytes(32, 128), tc_smem(3, 256));
 static_assert(TC_SMEM_MAX <= 227 * 1024, "tensor-core kernel shared memory");
 
 struct TcArgs {
@@ -65,18 +70,18 @@ struct TcArgs {
   float* gate_out;
   int* mask_count;
   WsHeader* hdr;
-  int* mflags;        // [4 * Mb]: epoch + 1 once an epilogue warp's 32 gt rows are out
-  __nv_bfloat16* gt;  // [Mb * 128][r]
+  int* mflags;        // [4 * Mb * BMT / 128]: epoch + 1 once an epilogue warp's 32 gt rows are out
+  __nv_bfloat16* gt;  // [Mb * BMT][r]
   int M, K, N, r, group;
   float b_g, tau;
-  int Mb, Nb;       // 128-token blocks, 256-channel blocks
+  int Mb, Nb;       // BMT-token blocks, 256-channel blocks
   int with_ec;      // projection tiles + EC k-steps
   int NE;           // projection tile width: 16 * ceil((r + 1) / 16)
   int ec_steps;     // ceil(r / 64)
   int gate_kind, gate_h;  // 0: scalar gate; 1: per-rank gamma(t) with bottleneck h
   const float *gw1, *gb1, *gw2, *gb2;
   float alpha;
-  int nst;                // ring stages (TC_STAGES, or one fewer with the rank gate)
+  int nst;                // ring stages
 };
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -200,7 +205,7 @@ __device__ __forceinline__ void dequant_tile(const uint8_t* psrc, uint8_t* bdst,
   }
 }
 
-template <bool GROUP>
+template <bool GROUP, int BMT>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_kernel(const __grid_constant__ TcArgs a, const __grid_constant__ CUtensorMap tm_x,
               const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_agt,
@@ -209,9 +214,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   // 1024-byte aligned base, derived from the shared array itself so that the
   // compiler keeps every access in the shared window (ld/st.shared)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* xs = smem;                                        // [STAGES][16 KB]
+  constexpr int NH = BMT / TC_BM;          // accumulators (M = 128 MMAs) per tile
+  constexpr int NBA = NH == 1 ? 2 : 1;      // accumulator buffers (TMEM holds 512 columns)
+  constexpr int XB = BMT * TC_BK * 2;       // x bytes of a stage
+  uint8_t* xs = smem;                                        // [NST][XB]
   const int NST = a.nst;
-  uint8_t* bs = smem + NST * TC_X_BYTES;                     // [NST][32 KB]
+  uint8_t* bs = smem + NST * XB;                             // [NST][32 KB]
   uint8_t* ps = bs + NST * TC_B_BYTES;                       // [NST][8 KB]
   uint64_t* bars = reinterpret_cast<uint64_t*>(ps + NST * TC_P_BYTES);
   uint64_t* full = bars;                     // TMA loads of a stage landed
@@ -233,7 +241,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&ready[s], 8);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NBA; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 4);
     }
@@ -268,18 +276,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         for (int k = 0; k < ti.steps && ok; ++k) {
           ok = mbar_wait(&empty[s], ph ^ 1, abort_flag, a.hdr);
           if (!ok) break;
-          uint8_t* xd = xs + s * TC_X_BYTES;
+          uint8_t* xd = xs + s * XB;
           uint8_t* bd = bs + s * TC_B_BYTES;
           uint8_t* pd = ps + s * TC_P_BYTES;
           if (ti.kind == 0) {
-            mbar_arrive_tx(&full[s], TC_X_BYTES + a.NE * 128);
-            tma_load_2d(smem_u32(xd), &tm_x, &full[s], k * TC_BK, ti.mb * TC_BM);
+            mbar_arrive_tx(&full[s], XB + a.NE * 128);
+            tma_load_2d(smem_u32(xd), &tm_x, &full[s], k * TC_BK, ti.mb * BMT);
             tma_load_2d(smem_u32(bd), &tm_agt, &full[s], k * TC_BK, 0);
           } else if (k < KT) {
             // warm L2 a few k-steps ahead so the shallow shared-memory ring
             // does not see the full HBM latency on every stage
             if (k + TC_PREFETCH < KT) {
-              tma_prefetch_2d(&tm_x, (k + TC_PREFETCH) * TC_BK, ti.mb * TC_BM);
+              tma_prefetch_2d(&tm_x, (k + TC_PREFETCH) * TC_BK, ti.mb * BMT);
               tma_prefetch_3d(&tm_w, 0, k + TC_PREFETCH, ti.nb * (TC_BN / 16));
             } else {
               // the tile's tail: warm its EC operands (L2 is coherent, so gt may
@@ -289,38 +297,39 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               if (j == 0 && a.with_ec)
                 for (int e = 0; e < a.ec_steps; ++e) {
                   tma_prefetch_2d(&tm_bpt, e * TC_BK, ti.nb * TC_BN);
-                  tma_prefetch_2d(&tm_gt, e * TC_BK, ti.mb * TC_BM);
+                  tma_prefetch_2d(&tm_gt, e * TC_BK, ti.mb * BMT);
                 }
               const int nt = tile + (int)gridDim.x;
               if (nt < ntiles) {
                 const TileInfo tn = tile_info(a, nt);
                 if (tn.kind == 1 && j < KT) {
-                  tma_prefetch_2d(&tm_x, j * TC_BK, tn.mb * TC_BM);
+                  tma_prefetch_2d(&tm_x, j * TC_BK, tn.mb * BMT);
                   tma_prefetch_3d(&tm_w, 0, j, tn.nb * (TC_BN / 16));
                 }
               }
             }
             if (k == 0)
               for (int pk = 1; pk < TC_PREFETCH && pk < KT; ++pk) {
-                tma_prefetch_2d(&tm_x, pk * TC_BK, ti.mb * TC_BM);
+                tma_prefetch_2d(&tm_x, pk * TC_BK, ti.mb * BMT);
                 tma_prefetch_3d(&tm_w, 0, pk, ti.nb * (TC_BN / 16));
               }
-            mbar_arrive_tx(&full[s], TC_X_BYTES + TC_P_BYTES);
-            tma_load_2d(smem_u32(xd), &tm_x, &full[s], k * TC_BK, ti.mb * TC_BM);
+            mbar_arrive_tx(&full[s], XB + TC_P_BYTES);
+            tma_load_2d(smem_u32(xd), &tm_x, &full[s], k * TC_BK, ti.mb * BMT);
             tma_load_3d(smem_u32(pd), &tm_w, &full[s], 0, k, ti.nb * (TC_BN / 16));
           } else {
             const int e = k - KT;
             if (e == 0) {
               // gated projection of this token block must be published
-              for (int qq = 0; qq < 4 && ok; ++qq) ok = wait_flag_eq(&a.mflags[4 * ti.mb + qq], epoch + 1, a.hdr);
+              for (int qq = 0; qq < 4 * NH && ok; ++qq)
+                ok = wait_flag_eq(&a.mflags[4 * NH * ti.mb + qq], epoch + 1, a.hdr);
               if (!ok) {
                 *abort_flag = 1;
                 break;
               }
               asm volatile("fence.proxy.async.global;" ::: "memory");
             }
-            mbar_arrive_tx(&full[s], TC_X_BYTES + TC_B_BYTES);
-            tma_load_2d(smem_u32(xd), &tm_gt, &full[s], e * TC_BK, ti.mb * TC_BM);
+            mbar_arrive_tx(&full[s], XB + TC_B_BYTES);
+            tma_load_2d(smem_u32(xd), &tm_gt, &full[s], e * TC_BK, ti.mb * BMT);
             tma_load_2d(smem_u32(bd), &tm_bpt, &full[s], e * TC_BK, ti.nb * TC_BN);
           }
           if (++s == NST) {
@@ -343,17 +352,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         ok = mbar_wait(&acc_empty[buf], aph[buf] ^ 1, abort_flag, a.hdr);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + buf * 256;
         const uint32_t idesc = ti.kind == 0 ? make_idesc(TC_BM, a.NE) : make_idesc(TC_BM, TC_BN);
         for (int k = 0; k < ti.steps && ok; ++k) {
           ok = mbar_wait(&ready[s], ph, abort_flag, a.hdr);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t ad = sw128_desc(smem_u32(xs + s * TC_X_BYTES));
           const uint64_t bd = sw128_desc(smem_u32(bs + s * TC_B_BYTES));
 #pragma unroll
-          for (int kk = 0; kk < TC_BK / 16; ++kk)
-            umma(d, ad + 2 * kk, bd + 2 * kk, idesc, (k > 0 || kk > 0) ? 1u : 0u);
+          for (int h = 0; h < NH; ++h) {
+            // rows 128 h .. 128 h + 127 of the x tile (8-row groups 1024 B apart)
+            const uint64_t ad = sw128_desc(smem_u32(xs + s * XB + h * TC_X_BYTES));
+            const uint32_t d = tmem_base + (uint32_t)(buf * NH + h) * 256;
+#pragma unroll
+            for (int kk = 0; kk < TC_BK / 16; ++kk)
+              umma(d, ad + 2 * kk, bd + 2 * kk, idesc, (k > 0 || kk > 0) ? 1u : 0u);
+          }
           umma_commit(&empty[s]);
           if (++s == NST) {
             s = 0;
@@ -363,7 +376,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (!ok) break;
         umma_commit(&acc_full[buf]);
         aph[buf] ^= 1;
-        buf ^= 1;
+        buf = buf + 1 == NBA ? 0 : buf + 1;
       }
     }
   } else if (warp < 6) {
@@ -395,9 +408,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], aph[buf], abort_flag, a.hdr));
       if (!ok) break;
       tc_fence_after();
+#pragma unroll 1
+      for (int h = 0; h < NH; ++h) {
       const int row = q * 32 + lane;
-      const int m = ti.mb * TC_BM + row;
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * 256;
+      const int m = ti.mb * BMT + h * TC_BM + row;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NH + h) * 256;
       if (ti.kind == 0) {
         // projection tile: columns 0..r-1 = t, column r = gate logit
         __nv_bfloat16* gdst = a.gt + (size_t)m * a.r;
@@ -483,7 +498,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         // one flag per epilogue warp (32 token rows), tagged with this launch's epoch
-        if (lane == 0) st_release_gpu(&a.mflags[4 * ti.mb + q], epoch + 1);
+        if (lane == 0) st_release_gpu(&a.mflags[4 * NH * ti.mb + 4 * h + q], epoch + 1);
       } else {
         const int n0 = ti.nb * TC_BN;
 #pragma unroll 1
@@ -512,10 +527,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         tc_fence_before();
       }
+      }  // accumulator halves
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
       aph[buf] ^= 1;
-      buf ^= 1;
+      buf = buf + 1 == NBA ? 0 : buf + 1;
     }
   } else {
     // ------------------------------------------------------------ dequant
@@ -577,25 +593,33 @@ TcPlan plan_tc(int M, int K, int N, int r, int group, int sm_count) {
   return p;
 }
 
-template <bool GROUP>
+template <bool GROUP, int BMT>
 static int launch_tc_t(const TcPlan& p, const TcArgs& a, const CUtensorMap* maps, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(tc_kernel<GROUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM_MAX);
+    attr_err = cudaFuncSetAttribute(tc_kernel<GROUP, BMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM_MAX);
   });
   if (attr_err != cudaSuccess) return set_cuda_error("cudaFuncSetAttribute(tc)", attr_err);
   const int ntiles = (a.with_ec ? a.Mb : 0) + a.Mb * a.Nb;
   const int grid = ntiles < p.grid ? ntiles : p.grid;
-  const size_t smem = a.gate_kind == 1 ? tc_smem(a.nst) + tc_gpar_bytes(a.gate_h, a.r) : tc_smem(a.nst);
-  tc_kernel<GROUP><<<grid, TC_THREADS, smem, st>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4]);
+  const size_t smem = tc_smem(a.nst, BMT) + (a.gate_kind == 1 ? tc_gpar_bytes(a.gate_h, a.r) : 0);
+  tc_kernel<GROUP, BMT><<<grid, TC_THREADS, smem, st>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4]);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPEAR_OK : set_cuda_error("tc kernel launch", e);
+}
+
+// Tile height: 256 tokens from M = 512 up (twice the tensor-core work per
+// dequantised tile and per ring round trip); 128 below, and with the rank
+// gate (whose parameters take the shared memory of a fourth stage).
+static int tc_tile_rows(int M, const LayerView& L, bool with_ec) {
+  return (M >= 512 && !(with_ec && L.r > 0 && L.gate_kind == 1)) ? 256 : 128;
 }
 
 int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, bool with_ec,
               WsHeader* hdr, int* mflags, __nv_bfloat16* gt, float* gate_out, int* mask_count, cudaStream_t st) {
   if (L.N % TC_BN) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "tensor-core path needs N %% 256 == 0 (N=%d)", L.N);
+  const int bmt = tc_tile_rows(M, L, with_ec);
   TcArgs a = {};
   a.scales = L.scales;
   a.y = y;
@@ -611,7 +635,7 @@ int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
   a.group = L.group;
   a.b_g = L.b_g;
   a.tau = L.tau;
-  a.Mb = p.m_blocks;
+  a.Mb = (M + bmt - 1) / bmt;
   a.Nb = p.n_blocks;
   a.with_ec = with_ec && L.r > 0;
   a.NE = 16 * ((a.r + 1 + 15) / 16);
@@ -623,17 +647,18 @@ int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
   a.gw2 = L.gw2;
   a.gb2 = L.gb2;
   a.alpha = L.alpha;
-  a.nst = a.gate_kind == 1 ? TC_STAGES - 1 : TC_STAGES;
+  a.nst = bmt == 256 ? 3 : (a.gate_kind == 1 ? TC_STAGES - 1 : TC_STAGES);
   CUtensorMap maps[5];
   memset(maps, 0, sizeof(maps));
-  bool ok = tmap_2d_bf16(&maps[0], x, L.K, M, TC_BK, TC_BM) && tmap_packed_box(&maps[1], L.w, L.K, L.N, 1, TC_BN / 16);
+  bool ok = tmap_2d_bf16(&maps[0], x, L.K, M, TC_BK, bmt) && tmap_packed_box(&maps[1], L.w, L.K, L.N, 1, TC_BN / 16);
   if (ok && a.with_ec) {
     ok = tmap_2d_bf16(&maps[2], L.agt, L.K, L.r + 1, TC_BK, a.NE) &&
          tmap_2d_bf16(&maps[3], L.bpt, L.r, L.N, TC_BK, TC_BN) &&
-         tmap_2d_bf16(&maps[4], gt, L.r, (uint64_t)p.m_blocks * TC_BM, TC_BK, TC_BM);
+         tmap_2d_bf16(&maps[4], gt, L.r, (uint64_t)a.Mb * bmt, TC_BK, bmt);
   }
   if (!ok) return set_error(SPEAR_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-  return L.group ? launch_tc_t<true>(p, a, maps, st) : launch_tc_t<false>(p, a, maps, st);
+  if (bmt == 256) return L.group ? launch_tc_t<true, 256>(p, a, maps, st) : launch_tc_t<false, 256>(p, a, maps, st);
+  return L.group ? launch_tc_t<true, 128>(p, a, maps, st) : launch_tc_t<false, 128>(p, a, maps, st);
 }
 
 }  // namespace spear
