@@ -115,6 +115,21 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
   asm volatile(
@@ -230,6 +245,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint32_t* tmem_base_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_holder + 1);
   float* gpar = reinterpret_cast<float*>(ps + NST * TC_P_BYTES + 1024);
+  // the output tile's 256 per-channel scales (epilogue warps), in the barrier block's second half
+  __half* esc = reinterpret_cast<__half*>(ps + NST * TC_P_BYTES + 512);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int epoch = *reinterpret_cast<volatile int*>(&a.hdr->epoch);
@@ -408,6 +425,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], aph[buf], abort_flag, a.hdr));
       if (!ok) break;
       tc_fence_after();
+      if (!GROUP && ti.kind == 1) {
+        // the tile's scales into shared memory once (the previous tile's
+        // readers are done: every epilogue warp passed the first barrier)
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const int et = threadIdx.x - 64;
+        reinterpret_cast<uint32_t*>(esc)[et] =
+            __ldg(reinterpret_cast<const uint32_t*>(a.scales + ti.nb * TC_BN) + et);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
 #pragma unroll 1
       for (int h = 0; h < NH; ++h) {
       const int row = q * 32 + lane;
@@ -502,27 +528,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       } else {
         const int n0 = ti.nb * TC_BN;
 #pragma unroll 1
-        for (int c0 = 0; c0 < TC_BN; c0 += 16) {
-          float v[16];
-          tmem_ld16(taddr + c0, v);
+        for (int c0 = 0; c0 < TC_BN; c0 += 32) {
+          float v[32];
+          tmem_ld32(taddr + c0, v);
           if (!GROUP) {
-            const uint4* sp = reinterpret_cast<const uint4*>(a.scales + n0 + c0);
-            const uint4 s0 = __ldg(sp), s1 = __ldg(sp + 1);
-            const __half* h0 = reinterpret_cast<const __half*>(&s0);
-            const __half* h1 = reinterpret_cast<const __half*>(&s1);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              v[i] *= __half2float(h0[i]);
-              v[8 + i] *= __half2float(h1[i]);
+            for (int i = 0; i < 32; i += 2) {
+              const float2 sc = __half22float2(*reinterpret_cast<const __half2*>(esc + c0 + i));
+              v[i] *= sc.x;
+              v[i + 1] *= sc.y;
             }
           }
           if (m < a.M) {
-            uint32_t pk[8];
+            uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
             uint4* dst = reinterpret_cast<uint4*>(a.y + (size_t)m * a.N + n0 + c0);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           }
         }
         tc_fence_before();
