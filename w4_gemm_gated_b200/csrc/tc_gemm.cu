@@ -60,9 +60,9 @@ constexpr int TC_SMEM = tc_smem(TC_STAGES, 128);
 // rank-gate parameters (W1 [h][r], W2 [r][h], b1 [h], b2 [r], fp32) after the barriers
 __host__ __device__ constexpr int tc_gpar_bytes(int h, int r) { return (2 * h * r + h + r) * 4; }
 constexpr int tc_max3(int a, int b, int c) { return a > b ? (a > c ? a : c) : (b > c ? b : c); }
-constexpr int TC_SMEM_MAX =
-    tc_max3(TC_SMEM, tc_smem(TC_STAGES - 1, 128) + tc_gpar_bytes(32, 128), tc_smem(3, 256));
-static_assert(TC_SMEM_MAX <= 227 * 1024, "tensor-core kernel shared memory");
+constexpr int TC_SMEM_MAX = 227 * 1024;  // the device's per-block limit
+static_assert(tc_max3(TC_SMEM, tc_smem(TC_STAGES - 1, 128) + tc_gpar_bytes(32, 128), tc_smem(3, 256)) <= TC_SMEM_MAX,
+              "tensor-core kernel shared memory");
 
 struct TcArgs {
   const __half* scales;
@@ -633,10 +633,12 @@ static int launch_tc_t(const TcPlan& p, const TcArgs& a, const CUtensorMap* maps
 }
 
 // Tile height: 256 tokens from M = 512 up (twice the tensor-core work per
-// dequantised tile and per ring round trip); 128 below, and with the rank
-// gate (whose parameters take the shared memory of a fourth stage).
+// dequantised tile and per ring round trip), when the rank gate's parameters,
+// if any, fit beside three stages; 128 otherwise.
 static int tc_tile_rows(int M, const LayerView& L, bool with_ec) {
-  return (M >= 512 && !(with_ec && L.r > 0 && L.gate_kind == 1)) ? 256 : 128;
+  if (M < 512) return 128;
+  const bool rank = with_ec && L.r > 0 && L.gate_kind == 1;
+  return (!rank || tc_smem(3, 256) + tc_gpar_bytes(L.gate_h, L.r) <= TC_SMEM_MAX) ? 256 : 128;
 }
 
 int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, bool with_ec,
