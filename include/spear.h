@@ -7,10 +7,13 @@
  * into a low-rank space with A, gates it per token and projects back with B,
  * on top of the 4-bit weight; fugumt.com abstract of arXiv 2606.11244: ECs
  * "modulated by per-token gates" over W4 per-channel weights), in the
- * row-vector scalar-gate form implemented here:
+ * row-vector form implemented here, with a scalar gate per token by default:
  *
  *     g_m = sigmoid(x_m . w_g + b_g)
  *     y_m = x_m . dequant(W4) + g_m * ((x_m . A) . B)
+ *
+ * or, per layer, the pages' per-rank gate gamma(x_m . A) (spear_layer's
+ * gate_kind, below).
  *
  *   x    M x K   bf16, row-major (token-major)
  *   W    K x N   logically; stored as N output channels x K int4 codes
@@ -32,7 +35,9 @@
  *     aborts or exits the process.
  *   - Shapes: K and N multiples of 128; r in {0, 16, 32, 64, 128}; group 0
  *     (one fp16 scale per output channel) or 128 (one fp16 scale per 128
- *     consecutive k and output channel); 1 <= M <= 65536.
+ *     consecutive k and output channel); 1 <= M <= 65536.  The tensor-core
+ *     paths also need N % 256 == 0 and the decode path (M <= 16) K % 128 == 0
+ *     (SPEAR_ERR_UNSUPPORTED_SHAPE otherwise).
  */
 #ifndef SPEAR_H_
 #define SPEAR_H_
