@@ -157,7 +157,7 @@ def time_oracle(target_s: float = 15.0, n_cols: int = 1376):
 # DRAM bytes per decode launch from the ncu captures summarised in profiles/
 # (dram__bytes_read.sum + dram__bytes_write.sum, one launch at M = 1 and at M = 16),
 # valid only while the decode kernel sources are the ones captured.
-DECODE_TRAFFIC = {"sources_sha1": "3caa4a3d34887b5e620b2005d122d336b2552828",
+DECODE_TRAFFIC = {"sources_sha1": "8e831b43424f917770705749463950a124d008ed",
                   "bytes_per_launch": {1: 24644864, 16: 24781568}}
 DECODE_SOURCES = ("w4_gemm_gated_b200/csrc/decode2.cu", "w4_gemm_gated_b200/csrc/common.cuh",
                   "w4_gemm_gated_b200/csrc/tma.cuh")

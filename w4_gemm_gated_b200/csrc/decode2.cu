@@ -17,8 +17,10 @@
 //
 // Streaming.  The producer warp issues TMA loads of units of at most 8 KB into
 // a shared-memory ring.  Weights, [A^T ; w_g] and the epilogue operands (B'
-// rows, scales) do not depend on the previous kernel in the stream, so they are
-// requested before the grid-dependency wait.
+// rows, scales) do not depend on the previous kernel in the stream: the
+// epilogue operands and the first two ring units are requested before the
+// grid-dependency wait, the rest of the ring after it (a full ring requested
+// early delays the activation load that follows the wait).
 //
 // Reduction, in a fixed order.  The 4 warp partials of a strip go through
 // shared memory to the reducer warp.  With CS > 1 the CTA partials go to the
