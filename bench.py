@@ -157,8 +157,8 @@ def time_oracle(target_s: float = 15.0, n_cols: int = 1376):
 # DRAM bytes per decode launch from the ncu captures summarised in profiles/
 # (dram__bytes_read.sum + dram__bytes_write.sum, one launch at M = 1 and at M = 16),
 # valid only while the decode kernel sources are the ones captured.
-DECODE_TRAFFIC = {"sources_sha1": "8e831b43424f917770705749463950a124d008ed",
-                  "bytes_per_launch": {1: 24644864, 16: 24781568}}
+DECODE_TRAFFIC = {"sources_sha1": "4b522b75ca9e1e065c18478861b7580446a3dbc5",
+                  "bytes_per_launch": {1: 24639488, 16: 24772608}}
 DECODE_SOURCES = ("w4_gemm_gated_b200/csrc/decode2.cu", "w4_gemm_gated_b200/csrc/common.cuh",
                   "w4_gemm_gated_b200/csrc/tma.cuh")
 

@@ -338,11 +338,107 @@ __device__ __forceinline__ void d2_ts_fetch(const unsigned long long* tt, unsign
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Rank gate (summary section 2.1 A) from the staged projection, one warp:
+// u = relu(W1 t + b1), gamma = sigmoid(W2 u + b2), gt[m][j] = bf16(alpha
+// gamma_j t[m][j]); padded tokens get zero rows.  Returns, on lane m of CTA 0
+// (report), token m's mean of gamma.  Kept out of line so that the scalar-gate
+// kernel body, and the inlining of its per-strip code, do not change with it.
+template <int MT>
+__device__ __noinline__ float d2_rank_gate(const unsigned long long* ts, __nv_bfloat16* gts, float* gsc,
+                                           const float* gpar, int M, int r, int h, float alpha, bool report,
+                                           int lane) {
+  auto tval = [&](int m, int row) {
+    return __uint_as_float((uint32_t)ts[((row >> 4) * MT + m) * 16 + (row & 15)]);
+  };
+  const int gs = r + 8;
+  const float* W1 = gpar;              // [h][r]
+  const float* W2 = gpar + h * r;      // [r][h]
+  const float* B1 = gpar + 2 * h * r;  // [h]
+  const float* B2 = B1 + h;            // [r]
+  // One warp builds this on every CTA's critical path, so the loops run over
+  // the live tokens only and every sum is four independent FMA chains.
+  // Hidden activations u[m][i]: M * h pairs; with fewer than 32 pairs, L
+  // adjacent lanes share a pair, each summing r / L of its products, and add
+  // them by a fixed shuffle tree.
+  const int P1 = M * h, r4 = r / 4;
+  int L = 1;
+  while (L < 4 && P1 * L * 2 <= 32) L *= 2;  // h >= 8, r >= 16: r4 / L >= 1
+  const int seg = r4 / L;
+  for (int base = 0; base < P1 * L; base += 32) {
+    const int idx = base + lane;
+    const int p = idx / L, sub = idx - p * L;
+    const bool live = p < P1;
+    const int m = live ? p / h : 0, i = live ? p - m * h : 0;
+    float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
+    if (live) {
+      const float4* w = reinterpret_cast<const float4*>(W1 + i * r) + sub * seg;
+      const int j0 = 4 * sub * seg;
+#pragma unroll 4
+      for (int q4 = 0; q4 < seg; ++q4) {
+        const float4 wv = w[q4];
+        v0 = fmaf(wv.x, tval(m, j0 + 4 * q4), v0);
+        v1 = fmaf(wv.y, tval(m, j0 + 4 * q4 + 1), v1);
+        v2 = fmaf(wv.z, tval(m, j0 + 4 * q4 + 2), v2);
+        v3 = fmaf(wv.w, tval(m, j0 + 4 * q4 + 3), v3);
+      }
+    }
+    float v = (v0 + v1) + (v2 + v3);
+    for (int off = L >> 1; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (live && sub == 0) gsc[m * 32 + i] = fmaxf(v + B1[i], 0.f);
+  }
+  __syncwarp();
+  // gamma and gt by (token, rank): M * r pairs, a multiple of 16; a batch of
+  // 32 pairs holds one token (r >= 32) or two (r = 16)
+  float gsum = 0.f;
+  for (int base = 0; base < M * r; base += 32) {
+    const int idx = base + lane;
+    const int m = idx / r, j = idx - m * r;
+    float gam = 0.f;
+    if (idx < M * r) {
+      const float4* w = reinterpret_cast<const float4*>(W2 + j * h);
+      const float4* u = reinterpret_cast<const float4*>(gsc + m * 32);
+      float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
+#pragma unroll
+      for (int i4 = 0; i4 < 8; ++i4) {
+        if (4 * i4 >= h) break;
+        const float4 wv = w[i4], uv = u[i4];
+        z0 = fmaf(wv.x, uv.x, z0);
+        z1 = fmaf(wv.y, uv.y, z1);
+        z2 = fmaf(wv.z, uv.z, z2);
+        z3 = fmaf(wv.w, uv.w, z3);
+      }
+      gam = sigmoidf_(B2[j] + ((z0 + z1) + (z2 + z3)));
+      gts[m * gs + j] = __float2bfloat16_rn(alpha * gam * tval(m, j));
+    }
+    if (report) {
+      // only CTA 0 reports the gate: this batch's gamma sum per token, by a
+      // fixed shuffle tree
+      float v = gam;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1)
+        if (off < r) v += __shfl_xor_sync(0xffffffffu, v, off);
+      const int m0 = base / r;
+      if (r >= 32) {
+        if (lane == m0) gsum += v;
+      } else {
+        const float va = __shfl_sync(0xffffffffu, v, 0), vb = __shfl_sync(0xffffffffu, v, 16);
+        if (lane == m0) gsum += va;
+        if (lane == m0 + 1) gsum += vb;
+      }
+    }
+  }
+  // the padded tokens' rows of gt are zero
+  for (int idx = lane; idx < (MT - M) * (r / 2); idx += 32) {
+    const int m = M + idx / (r / 2), j = 2 * (idx - (idx / (r / 2)) * (r / 2));
+    *reinterpret_cast<uint32_t*>(gts + m * gs + j) = 0u;
+  }
+  return gsum / (float)r;
+}
+
 // Gate and gt from the staged projection (one warp).  Scalar gate:
-// g_m = sigmoid(t[m][r] + b_g), gt[m][j] = bf16(g_m t[m][j]).  Rank gate
-// (summary section 2.1 A): u = relu(W1 t + b1), gamma = sigmoid(W2 u + b2),
-// gt[m][j] = bf16(alpha gamma_j t[m][j]), and the reported gate is the mean of
-// gamma.  CTA 0 also writes the gate outputs and the mask count.
+// g_m = sigmoid(t[m][r] + b_g), gt[m][j] = bf16(g_m t[m][j]); rank gate: see
+// d2_rank_gate, with the mean of gamma as the reported gate.  CTA 0 also writes
+// the gate outputs and the mask count.
 template <int MT>
 __device__ void d2_build_gt(const D2Args& a, const unsigned long long* ts, __nv_bfloat16* gts, float* gsc,
                             const float* gpar, int lane) {
@@ -352,69 +448,7 @@ __device__ void d2_build_gt(const D2Args& a, const unsigned long long* ts, __nv_
   const int gs = a.r + 8;
   float g;  // lane m: token m's gate
   if (a.gate_kind == 1) {
-    const int h = a.gate_h, r = a.r;
-    const float* W1 = gpar;              // [h][r]
-    const float* W2 = gpar + h * r;      // [r][h]
-    const float* B1 = gpar + 2 * h * r;  // [h]
-    const float* B2 = B1 + h;            // [r]
-    // hidden activations of the live tokens
-    for (int idx = lane; idx < MT * h; idx += 32) {
-      const int m = idx / h, i = idx - m * h;
-      float v = 0.f;
-      if (m < a.M) {
-        v = B1[i];
-        const float4* w = reinterpret_cast<const float4*>(W1 + i * r);
-#pragma unroll 4
-        for (int j4 = 0; j4 < r / 4; ++j4) {
-          const float4 wv = w[j4];
-          v = fmaf(wv.x, tval(m, 4 * j4), v);
-          v = fmaf(wv.y, tval(m, 4 * j4 + 1), v);
-          v = fmaf(wv.z, tval(m, 4 * j4 + 2), v);
-          v = fmaf(wv.w, tval(m, 4 * j4 + 3), v);
-        }
-        v = fmaxf(v, 0.f);
-      }
-      gsc[m * 32 + i] = v;
-    }
-    __syncwarp();
-    // gamma and gt by (token, rank); MT * r is a multiple of 32, and a batch of
-    // 32 pairs holds one token (r >= 32) or two (r = 16)
-    float gsum = 0.f;
-    for (int base = 0; base < MT * r; base += 32) {
-      const int idx = base + lane;
-      const int m = idx / r, j = idx - m * r;
-      float gam = 0.f, o = 0.f;
-      if (m < a.M) {
-        float z = B2[j];
-        const float4* w = reinterpret_cast<const float4*>(W2 + j * h);
-#pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-          if (4 * i4 >= h) break;
-          const float4 wv = w[i4];
-          z = fmaf(wv.x, gsc[m * 32 + 4 * i4], z);
-          z = fmaf(wv.y, gsc[m * 32 + 4 * i4 + 1], z);
-          z = fmaf(wv.z, gsc[m * 32 + 4 * i4 + 2], z);
-          z = fmaf(wv.w, gsc[m * 32 + 4 * i4 + 3], z);
-        }
-        gam = sigmoidf_(z);
-        o = a.alpha * gam * tval(m, j);
-      }
-      gts[m * gs + j] = __float2bfloat16_rn(o);
-      // this batch's gamma sum per token, by a fixed shuffle tree
-      float v = gam;
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1)
-        if (off < r) v += __shfl_xor_sync(0xffffffffu, v, off);
-      const int m0 = base / r;
-      if (r >= 32) {
-        if (lane == m0) gsum += v;
-      } else {
-        const float v0 = __shfl_sync(0xffffffffu, v, 0), v1 = __shfl_sync(0xffffffffu, v, 16);
-        if (lane == m0) gsum += v0;
-        if (lane == m0 + 1) gsum += v1;
-      }
-    }
-    g = gsum / (float)r;
+    g = d2_rank_gate<MT>(ts, gts, gsc, gpar, a.M, a.r, a.gate_h, a.alpha, blockIdx.x == 0, lane);
   } else {
     g = lane < MT ? sigmoidf_(tval(lane, a.r) + a.b_g) : 0.f;
     const int half = a.r / 2;
