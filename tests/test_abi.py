@@ -225,3 +225,37 @@ def test_rank_gate_validation_before_launch(S, kw, code):
     rc = S.F["spear_linear_forward"](ctypes.byref(st), 0x50000, 4, 0x60000, 0x70000, 1 << 30, None, None, None)
     assert rc == code, S.F["spear_last_error"]().decode()
     assert S.F["spear_last_error"]().decode()
+
+
+def test_binding_struct_and_constants_match_the_header(S, tmp_path):
+    """The ctypes mirror of spear_layer has the C layout (every field offset and
+    the size, as gcc lays out include/spear.h), and the binding's status, path
+    and gate constants equal the header's enumerators."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not found")
+    fields = [name for name, _ in S.LayerStruct._fields_]
+    consts = {"OK": "SPEAR_OK"}
+    consts.update({n: "SPEAR_" + n for n in dir(S)
+                   if re.fullmatch(r"(ERR|PATH|GATE)_[A-Z_]+", n) and isinstance(getattr(S, n), int)})
+    lines = ['#include <stdio.h>', '#include "spear.h"', "int main(void) {",
+             '  printf("size %zu\\n", sizeof(spear_layer));']
+    lines += [f'  printf("field {f} %zu\\n", offsetof(spear_layer, {f}));' for f in fields]
+    lines += [f'  printf("const {py} %d\\n", (int){c});' for py, c in sorted(consts.items())]
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([gcc, "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    # tokens: "size" v, then ("field" | "const") name v triples
+    size = int(out[1])
+    got = {(out[i], out[i + 1]): int(out[i + 2]) for i in range(2, len(out), 3)}
+    assert size == ctypes.sizeof(S.LayerStruct)
+    for f in fields:
+        assert got[("field", f)] == getattr(S.LayerStruct, f).offset, f
+    assert len(consts) >= 14
+    for py in consts:
+        assert got[("const", py)] == getattr(S, py), py
