@@ -259,3 +259,40 @@ def test_binding_struct_and_constants_match_the_header(S, tmp_path):
     assert len(consts) >= 14
     for py in consts:
         assert got[("const", py)] == getattr(S, py), py
+
+
+def _c_kind(decl: str) -> str:
+    """Kind of a C parameter or return type as the binding must pass it."""
+    d = decl.strip()
+    if "*" in d:
+        return "ptr"
+    t = re.sub(r"\b(const|unsigned|signed)\b", "", d).split()
+    base = t[0] if t else ""
+    return {"int": "int", "size_t": "size_t", "float": "float", "void": "void"}.get(base, base)
+
+
+def _ctypes_kind(t) -> str:
+    if t is None:
+        return "void"
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "ptr"
+    return {ctypes.c_int: "int", ctypes.c_size_t: "size_t", ctypes.c_float: "float"}.get(t, repr(t))
+
+
+def test_binding_prototypes_match_the_header(S):
+    """Every header function's parameters (count and kind: pointer, int, size_t,
+    float) and return kind equal the binding's ctypes prototype."""
+    src = open(os.path.join(ROOT, "include", "spear.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    decls = re.findall(r"^\s*((?:const\s+)?[A-Za-z_0-9]+\s*\**)\s*\**\s*(spear_[A-Za-z_0-9]+)\s*\(([^)]*)\)\s*;",
+                       src, flags=re.M)
+    assert len(decls) == len(_header_functions())
+    for ret, name, params in decls:
+        # the pointer star may sit with the name ("const char* spear_x(") or the type
+        ret_kind = "ptr" if re.search(r"\*\s*" + name, src) or "*" in ret else _c_kind(ret)
+        args = [p for p in (x.strip() for x in params.split(",")) if p and p != "void"]
+        want = [_c_kind(p) for p in args]
+        sig = S.EXPORTS[name]
+        got = [_ctypes_kind(t) for t in sig[1:]]
+        assert got == want, (name, got, want)
+        assert _ctypes_kind(sig[0]) == ret_kind, (name, sig[0], ret)
