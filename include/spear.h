@@ -224,7 +224,7 @@ int spear_read_status(void* ws, int* device_status, void* stream);
  * allocation would synchronise the device, or plugin hosts that pass only
  * input and output buffers.
  * Same result as spear_linear_forward_path(..., SPEAR_PATH_DECODE, ...), but
- * the scratch lives in a 16 KB device array inside the library instead of a
+ * the scratch lives in a 40 KB device array inside the library instead of a
  * caller workspace.  Limit: 1 <= M <= 16 (larger M returns
  * SPEAR_ERR_UNSUPPORTED_SHAPE); every layer shape of the decode path.
  * No device memory is allocated or freed.  The first call on a device looks
