@@ -216,6 +216,22 @@ int spear_linear_forward_path(const spear_layer* layer, const uint16_t* x, int M
  * *device_status receives SPEAR_OK or the first device-side error code. */
 int spear_read_status(void* ws, int* device_status, void* stream);
 
+/* ---- failure injection (tests of the device-side error path only) -----------
+ * Makes one bounded device wait impossible to satisfy in the launches that
+ * follow, until called again with kernel 0: the wait expects a publication
+ * tag that no launch writes, and gives up after wait_cycles SM clock cycles
+ * instead of about a second.
+ *   kernel 1: the decode kernel's wait for the published EC rows;
+ *   kernel 2: the tensor-core kernel's wait for the gated projection.
+ * The launch then reports SPEAR_ERR_TIMEOUT in its status word (workspace, or
+ * the allocation-free call's array), every role of the kernel stops at its
+ * next check, waits for the copies it has in flight and exits; y is left
+ * unspecified.  No fault, trap or unbounded wait is involved.  As after any
+ * timeout, re-initialise the workspace (spear_workspace_init) before the next
+ * call.  Process-wide, not thread-safe against concurrent layer calls.
+ * SPEAR_ERR_INVALID_ARG for another kernel value or wait_cycles < 1. */
+int spear_test_inject_timeout(int kernel, long long wait_cycles);
+
 /* ---- allocation-free decode call ---------------------------------------------
  * Not part of the method on the pages (they have no counterpart): an
  * interface for callers that cannot allocate device memory where they run
@@ -227,15 +243,26 @@ int spear_read_status(void* ws, int* device_status, void* stream);
  * the scratch lives in a 40 KB device array inside the library instead of a
  * caller workspace.  Limit: 1 <= M <= 16 (larger M returns
  * SPEAR_ERR_UNSUPPORTED_SHAPE); every layer shape of the decode path.
- * No device memory is allocated or freed.  The first call on a device looks
- * up the array's device address (cudaGetSymbolAddress) and caches it, so
- * make that first call before any stream capture.  Each call clears the
+ * x, y: 16-byte aligned; gate_out, mask_count: 4-byte aligned (or NULL).
+ * No device memory is allocated or freed.  Every call looks up the array's
+ * device address (cudaGetSymbolAddress) on the current device; the first
+ * lookup on a device may load the library's device code, so make the first
+ * call on each device before any stream capture.  Each call clears the
  * array's launch header on `stream` before its kernel.  The array is shared
  * by all calls on a device: calls whose executions may overlap on the GPU
- * (other streams, unordered host threads) race and must not be issued. */
+ * (other streams, unordered host threads) race and must not be issued.
+ * Device-side failures (a bounded wait that expired) go to the array's own
+ * status word, which later calls do not clear: read it with
+ * spear_read_status_noalloc. */
 int spear_linear_forward_decode_noalloc(const spear_layer* layer, const uint16_t* x, int M,
                                         uint16_t* y, float* gate_out, int* mask_count,
                                         void* stream);
+
+/* Synchronise stream, then read and clear the status word of the
+ * allocation-free call's array on the current device.  *device_status
+ * receives SPEAR_OK or the first device-side error code recorded since the
+ * last read. */
+int spear_read_status_noalloc(int* device_status, void* stream);
 
 /* ---- a-7: dispatcher ----------------------------------------------------------
  * Phase-aware choice between the fused and the unfused EC path (SPEAR,
@@ -243,8 +270,9 @@ int spear_linear_forward_decode_noalloc(const spear_layer* layer, const uint16_t
  * adaptatif sensible a la phase": decode fuses the EC into the low-bit GEMM,
  * prefill runs it as a separate kernel; the choice here comes from measured
  * kernel times, the pages' latency tables of section 2.2 C).
- * The table is keyed by (K, N, r, group, M bucket); M buckets are powers of
- * two (M rounded up).  Before tuning: DECODE for M <= 16, else FUSED. */
+ * The table is keyed by (K, N, r, group, gate form, bottleneck width, M
+ * bucket); M buckets are powers of two (M rounded up).  Before tuning: DECODE
+ * for M <= 16, else FUSED. */
 int spear_dispatch_choice(const spear_layer* layer, int M);
 
 /* Time every applicable path for each M in Ms[0..nM) with CUDA events
@@ -260,8 +288,13 @@ int spear_dispatch_tune(const spear_layer* layer, const int* Ms, int nM,
                         void* flush, size_t flush_bytes, int reps, float* times_us,
                         void* stream);
 
-/* Set one table entry by hand (path is a SPEAR_PATH_* other than AUTO). */
+/* Set one table entry by hand (path is a SPEAR_PATH_* other than AUTO), for
+ * a layer with the scalar gate (or without an EC). */
 int spear_dispatch_set(int K, int N, int r, int group, int M, int path);
+/* Set the entry of this layer's full key -- shape, scale kind and gate form
+ * (a rank-gate layer has entries of its own, per bottleneck width) -- at M's
+ * bucket, with its measured time in microseconds (us < 0: not measured). */
+int spear_dispatch_set_layer(const spear_layer* layer, int M, int path, float us);
 /* Set one table entry with its measured time in microseconds (us >= 0).
  * Entries made by spear_dispatch_set carry no time; spear_dispatch_tune
  * records the median of the path it picks. */
@@ -271,9 +304,14 @@ int spear_dispatch_set_time(int K, int N, int r, int group, int M, int path, flo
 int spear_dispatch_time_us(const spear_layer* layer, int M, float* us);
 /* Forget every table entry. */
 void spear_dispatch_clear(void);
-/* Save / load the table as text (host file path).  Lines are
- * "K N r group M_bucket path time_us"; a line without the time loads as
- * not measured. */
+/* Save / load the table as text (host file path).  The first line names the
+ * device the times were measured on ("# spear dispatch table v3 sms=<count>
+ * device=<name>"); loading a table made on another device (name or SM count)
+ * fails with SPEAR_ERR_INVALID_ARG and leaves the table unchanged.  Entry
+ * lines are "K N r group gate_kind gate_hidden M_bucket path time_us"
+ * (time -1 or absent: not measured).  A file without the device line is read
+ * in the earlier format, "K N r group M_bucket path [time_us]", as
+ * scalar-gate entries. */
 int spear_dispatch_save(const char* path);
 int spear_dispatch_load(const char* path);
 

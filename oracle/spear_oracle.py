@@ -21,7 +21,7 @@ with x (M x K), W logically K x N stored per output channel, A (K x r),
 B (r x N), w_g (K), b_g a scalar.  Everything is evaluated in float64 from
 the exact values of the bf16 / fp16 inputs.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
   * the pages' global strength alpha is 1 (folded into B);
   * quantiser: symmetric RTN; scale s = fp16_rne(max|w| / 7) computed in
     fp32, saturated to 65504; a scale that is 0 becomes 1.0 with all codes 0;

@@ -156,6 +156,85 @@ def test_dispatch_times_save_load_and_v1_lines(S, tmp_path):
     S.dispatch_clear()
 
 
+def _rank_layer(S, h=16, **kw):
+    st = _layer(S, **kw)
+    st.gate_kind = S.GATE_RANK_MLP
+    st.gate_hidden = h
+    st.gate_w1, st.gate_b1, st.gate_w2, st.gate_b2 = 0x80000, 0x90000, 0xA0000, 0xB0000
+    st.gate_alpha = 1.0
+    return st
+
+
+def test_dispatch_key_separates_gate_forms(S, tmp_path):
+    # a scalar-gate and a rank-gate layer of the same (K, N, r, group) have
+    # entries of their own, per bottleneck width, and the SLO picker reads the
+    # entry of each layer's own gate form
+    S.dispatch_clear()
+    sc = _layer(S, K=4096, N=4096, r=64)
+    rk = _rank_layer(S, K=4096, N=4096, r=64, h=16)
+    rk32 = _rank_layer(S, K=4096, N=4096, r=64, h=32)
+    S.dispatch_set_layer(sc, 256, S.PATH_FUSED, 40.0)
+    S.dispatch_set_layer(rk, 256, S.PATH_SEMIFUSED, 90.0)
+    choice = S.F["spear_dispatch_choice"]
+    assert choice(ctypes.byref(sc), 256) == S.PATH_FUSED
+    assert choice(ctypes.byref(rk), 256) == S.PATH_SEMIFUSED
+    assert choice(ctypes.byref(rk32), 256) == S.PATH_FUSED          # no entry: the default
+    assert S.dispatch_time_us(sc, 200) == pytest.approx(40.0)
+    assert S.dispatch_time_us(rk, 200) == pytest.approx(90.0)
+    with pytest.raises(S.SpearError):
+        S.dispatch_time_us(rk32, 200)
+    # the scalar-gate setter writes the scalar-gate entry only
+    S.dispatch_set_time(4096, 4096, 64, 0, 256, S.PATH_UNFUSED, 55.0)
+    assert S.dispatch_time_us(sc, 256) == pytest.approx(55.0)
+    assert S.dispatch_time_us(rk, 256) == pytest.approx(90.0)
+    arr = (ctypes.POINTER(S.LayerStruct) * 1)
+    out, pred = ctypes.c_int(-1), ctypes.c_float(-1.0)
+    chunks = (ctypes.c_int * 1)(256)
+    rc = S.F["spear_slo_chunk"](arr(ctypes.pointer(sc)), 1, 0, 60.0, 0.0, chunks, 1, ctypes.byref(out),
+                                ctypes.byref(pred))
+    assert rc == S.OK and out.value == 256 and pred.value == pytest.approx(55.0)
+    rc = S.F["spear_slo_chunk"](arr(ctypes.pointer(rk)), 1, 0, 60.0, 0.0, chunks, 1, ctypes.byref(out),
+                                ctypes.byref(pred))
+    assert rc == S.OK and out.value == 0                          # 90 us does not fit 60 us
+    # the gate fields survive a save and load
+    p = str(tmp_path / "lut.txt")
+    S.dispatch_save(p)
+    S.dispatch_clear()
+    S.dispatch_load(p)
+    assert S.dispatch_time_us(rk, 256) == pytest.approx(90.0)
+    assert S.dispatch_time_us(sc, 256) == pytest.approx(55.0)
+    S.dispatch_clear()
+
+
+def test_timeout_injection_validates_its_arguments(S):
+    assert S.F["spear_test_inject_timeout"](3, 1000) == S.ERR_INVALID_ARG
+    assert S.F["spear_test_inject_timeout"](1, 0) == S.ERR_INVALID_ARG
+    assert S.F["spear_test_inject_timeout"](-1, 1000) == S.ERR_INVALID_ARG
+    assert S.F["spear_test_inject_timeout"](0, 0) == S.OK
+
+
+def test_dispatch_table_from_another_device_is_refused(S, tmp_path):
+    S.dispatch_clear()
+    sc = _layer(S, K=4096, N=4096, r=64)
+    S.dispatch_set_layer(sc, 64, S.PATH_FUSED, 30.0)
+    p = tmp_path / "lut.txt"
+    S.dispatch_save(str(p))
+    lines = p.read_text().splitlines()
+    assert lines[0].startswith("# spear dispatch table v3 sms=")
+    S.dispatch_clear()
+    S.dispatch_load(str(p))                                       # same device: accepted
+    assert S.dispatch_time_us(sc, 64) == pytest.approx(30.0)
+    S.dispatch_clear()
+    other = tmp_path / "other.txt"
+    other.write_text("# spear dispatch table v3 sms=7 device=Some Other GPU\n" + "\n".join(lines[1:]) + "\n")
+    with pytest.raises(S.SpearError):
+        S.dispatch_load(str(other))
+    assert "Some Other GPU" in S.F["spear_last_error"]().decode()
+    with pytest.raises(S.SpearError):                              # nothing was loaded
+        S.dispatch_time_us(sc, 64)
+    S.dispatch_clear()
+
+
 def _brute_slo(times, decode, slo, overhead, chunks):
     """Enumerate every candidate: predicted = overhead + sum of the layers'
     tabled times at the power-of-two bucket of decode + chunk."""
@@ -268,6 +347,8 @@ def _c_kind(decl: str) -> str:
         return "ptr"
     t = re.sub(r"\b(const|unsigned|signed)\b", "", d).split()
     base = t[0] if t else ""
+    if base == "long" and len(t) > 1 and t[1] == "long":
+        return "long long"
     return {"int": "int", "size_t": "size_t", "float": "float", "void": "void"}.get(base, base)
 
 
@@ -276,7 +357,8 @@ def _ctypes_kind(t) -> str:
         return "void"
     if t in (ctypes.c_void_p, ctypes.c_char_p) or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
         return "ptr"
-    return {ctypes.c_int: "int", ctypes.c_size_t: "size_t", ctypes.c_float: "float"}.get(t, repr(t))
+    return {ctypes.c_int: "int", ctypes.c_size_t: "size_t", ctypes.c_float: "float",
+            ctypes.c_longlong: "long long"}.get(t, repr(t))
 
 
 def test_binding_prototypes_match_the_header(S):

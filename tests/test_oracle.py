@@ -132,6 +132,36 @@ def test_linear_matches_bruteforce(group):
     assert np.allclose(y, yb, rtol=1e-12, atol=1e-12)
 
 
+def test_linear_matches_bruteforce_several_scale_groups():
+    # K = 384 with group 128: three scale groups per channel, each from its own
+    # block of 128 k, so a dequantiser that used one group's scale for another
+    # (or the per-channel layout) disagrees with the loop
+    L, q, s = _small_layer(128, seed=11, M=3, K=384, N=16, r=3, b_g=-0.5)
+    assert s.shape == (3, 16)
+    assert not np.array_equal(s[0], s[1]) and not np.array_equal(s[1], s[2])
+    y, g = O.linear(L.x, q, s, 128, L.A, L.B, L.w_g, L.b_g)
+    yb = O.linear_bruteforce(L.x, q, s, 128, L.A, L.B, L.w_g, L.b_g)
+    assert np.allclose(y, yb, rtol=1e-12, atol=1e-12)
+
+
+def test_one_hot_token_closed_form_several_scale_groups():
+    # x = e_k with k in the second and third scale groups: y[n] picks the scale
+    # of k's own group, s[k // 128, n]
+    L, q, s = _small_layer(128, seed=12, M=1, K=384, N=16, r=2)
+    A = O.bf16_to_f64(L.A)
+    B = O.bf16_to_f64(L.B)
+    wg = O.bf16_to_f64(L.w_g)
+    s64 = s.astype(np.float64)
+    for k in [128, 200, 255, 256, 383]:
+        x = np.zeros((1, L.K), dtype=np.uint16)
+        x[0, k] = 0x3F80                            # bf16 1.0
+        y, g = O.linear(x, q, s, 128, L.A, L.B, L.w_g, L.b_g)
+        gk = 1.0 / (1.0 + math.exp(-(wg[k] + L.b_g)))
+        for n in range(L.N):
+            ec = sum(A[k, j] * B[j, n] for j in range(L.r))
+            assert y[0, n] == pytest.approx(s64[k // 128, n] * q[n, k] + gk * ec, rel=1e-13, abs=1e-15)
+
+
 @pytest.mark.parametrize("group", [0, 128])
 def test_one_hot_token_closed_form(group):
     # x = e_k: y[n] = s(k, n) * q[n, k] + sigmoid(w_g[k] + b_g) * sum_j A[k, j] B[j, n]

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libspear.so")
-SOURCES = ["api.cu", "pack.cu", "decode.cu", "decode2.cu", "ec.cu", "tc_gemm.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "pack.cu", "decode.cu", "decode2.cu", "decode3.cu", "ec.cu", "tc_gemm.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h", "tma.cuh"]
 
 NVCC_FLAGS = [

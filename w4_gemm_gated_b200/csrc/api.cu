@@ -33,6 +33,13 @@ int set_cuda_error(const char* what, cudaError_t e) {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+static std::mutex g_fault_mu;
+static TestFault g_fault = {0, 0};
+TestFault test_fault() {
+  std::lock_guard<std::mutex> lk(g_fault_mu);
+  return g_fault;
+}
+
 static int sm_count() {
   static std::mutex mu;
   static std::map<int, int> cache;
@@ -175,7 +182,10 @@ static WsLayout ws_layout(const LayerView& L, int M_max) {
 // ---------------------------------------------------------------------------
 // dispatch table
 // ---------------------------------------------------------------------------
-using DKey = std::tuple<int, int, int, int, int>;  // K, N, r, group, M bucket
+// K, N, r, group, gate kind, gate bottleneck width, M bucket: a scalar-gate and a
+// rank-gate layer of the same shape run at different speeds, so they have
+// separate entries (gate fields are 0 for the scalar gate and without an EC)
+using DKey = std::tuple<int, int, int, int, int, int, int>;
 static std::mutex g_dmu;
 struct DEntry {
   int path;
@@ -189,6 +199,24 @@ static int m_bucket(int M) {
   return b;
 }
 
+static DKey dkey(const LayerView& L, int M) {
+  const int gk = L.r > 0 ? L.gate_kind : 0;
+  return DKey(L.K, L.N, L.r, L.group, gk, gk ? L.gate_h : 0, m_bucket(M));
+}
+
+// The device a table is measured on: its name and multiprocessor count.
+static std::string device_ident(int* sms_out) {
+  int dev = 0;
+  cudaDeviceProp prop;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+    cudaGetLastError();
+    *sms_out = 0;
+    return "no-device";
+  }
+  *sms_out = prop.multiProcessorCount;
+  return prop.name;
+}
+
 static int default_path(const LayerView& L, int M) {
   (void)L;
   return M <= 16 ? SPEAR_PATH_DECODE : SPEAR_PATH_FUSED;
@@ -197,7 +225,7 @@ static int default_path(const LayerView& L, int M) {
 static int choose_path(const LayerView& L, int M) {
   {
     std::lock_guard<std::mutex> lk(g_dmu);
-    auto it = g_table.find(DKey(L.K, L.N, L.r, L.group, m_bucket(M)));
+    auto it = g_table.find(dkey(L, M));
     if (it != g_table.end()) {
       const int p = it->second.path;
       if (!(p == SPEAR_PATH_DECODE && M > 16)) return p;
@@ -250,50 +278,45 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
   __nv_bfloat16* gt = reinterpret_cast<__nv_bfloat16*>(ws + wl.gt);
   float* part = reinterpret_cast<float*>(ws + wl.part);
   const int sms = sm_count();
-  if (path == SPEAR_PATH_DECODE) {
-    if (M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs M <= 16 (M=%d)", M);
-    if (!decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind, L.gate_h))
-      return launch_decode2(L, x, M, y, hdr, tbuf, gate_out, mask_count, false, st);
-    if (L.gate_kind)
-      return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: the rank gate needs the main decode kernel (%s)",
-                       decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind, L.gate_h));
-    DecodePlan p = plan_decode(M, L.K, L.N, L.r, L.group, sms);
+  // A decode-path launch (M <= 16) of layer LL: the kernel without a serial
+  // reducer where it runs the shape, else the earlier decode kernel, else the
+  // cluster split-K kernel (long or ragged K).
+  auto decode_launch = [&](const LayerView& LL, float* go, int* mc, bool ec_only) -> int {
+    if (!decode3_unsupported(M, LL.K, LL.N, LL.r, LL.group, LL.gate_kind, LL.gate_h))
+      return launch_decode3(LL, x, M, y, hdr, tbuf, go, mc, ec_only, st);
+    if (!decode2_unsupported(M, LL.K, LL.N, LL.r, LL.gate_kind, LL.gate_h))
+      return launch_decode2(LL, x, M, y, hdr, tbuf, go, mc, ec_only, st);
+    if (LL.r > 0 && LL.gate_kind)
+      return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: the rank gate needs the main decode kernels (%s)",
+                       decode2_unsupported(M, LL.K, LL.N, LL.r, LL.gate_kind, LL.gate_h));
+    DecodePlan p = plan_decode(M, LL.K, LL.N, LL.r, LL.group, sms);
     const char* why = check_decode_plan(p);
     if (why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", why);
-    return launch_decode(p, L, x, M, y, hdr, tbuf, gt, gate_out, mask_count, false, st);
+    return launch_decode(p, LL, x, M, y, hdr, tbuf, gt, go, mc, ec_only, st);
+  };
+  LayerView L0 = L;  // the same layer with the EC disabled
+  L0.r = 0;
+  L0.agt = nullptr;
+  L0.bpt = nullptr;
+  L0.gate_kind = 0;
+  if (path == SPEAR_PATH_DECODE) {
+    if (M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs M <= 16 (M=%d)", M);
+    return decode_launch(L, gate_out, mask_count, false);
   }
   if (path == SPEAR_PATH_UNFUSED) {
-    LayerView L0 = L;
-    L0.r = 0;
-    L0.agt = nullptr;
-    L0.bpt = nullptr;
-    L0.gate_kind = 0;
     int rc;
-    if (M <= 16 && !decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind, L.gate_h)) {
-      rc = launch_decode2(L0, x, M, y, hdr, tbuf, L.r > 0 ? nullptr : gate_out, L.r > 0 ? nullptr : mask_count,
-                          false, st);
+    if (M <= 16) {
+      if (L.r > 0 && L.gate_kind && decode3_unsupported(M, L.K, L.N, L.r, L.group, L.gate_kind, L.gate_h) &&
+          decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind, L.gate_h))
+        return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "unfused path at M <= 16: the rank gate needs the main decode kernels");
+      rc = decode_launch(L0, L.r > 0 ? nullptr : gate_out, L.r > 0 ? nullptr : mask_count, false);
       if (rc || L.r == 0) return rc;
-      // the separate EC launch: same kernel in EC-only mode, y += g (t . B) in place
-      return launch_decode2(L, x, M, y, hdr, tbuf, gate_out, mask_count, true, st);
-    } else if (M <= 16) {
-      if (L.gate_kind)
-        return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "unfused path at M <= 16: the rank gate needs the main decode kernel");
-      DecodePlan p = plan_decode(M, L.K, L.N, 0, L.group, sms);
-      const char* why = check_decode_plan(p);
-      if (why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", why);
-      rc = launch_decode(p, L0, x, M, y, hdr, tbuf, gt, L.r > 0 ? nullptr : gate_out,
-                         L.r > 0 ? nullptr : mask_count, false, st);
-      if (rc || L.r == 0) return rc;
-      // the separate EC launch: same kernel in EC-only mode, y += g (t . B) in place
-      DecodePlan pe = plan_decode(M, L.K, L.N, L.r, L.group, sms);
-      why = check_decode_plan(pe);
-      if (why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", why);
-      return launch_decode(pe, L, x, M, y, hdr, tbuf, gt, gate_out, mask_count, true, st);
-    } else {
-      TcPlan p = plan_tc(M, L.K, L.N, 0, L.group, sms);
-      rc = launch_tc(p, L0, x, M, y, false, hdr, tcflags, gt, L.r > 0 ? nullptr : gate_out,
-                     L.r > 0 ? nullptr : mask_count, st);
+      // the separate EC launch: a decode kernel in EC-only mode, y += g (t . B) in place
+      return decode_launch(L, gate_out, mask_count, true);
     }
+    TcPlan p = plan_tc(M, L.K, L.N, 0, L.group, sms);
+    rc = launch_tc(p, L0, x, M, y, false, hdr, tcflags, gt, L.r > 0 ? nullptr : gate_out,
+                   L.r > 0 ? nullptr : mask_count, st);
     if (rc || L.r == 0) return rc;
     // the separate EC kernel: projection and gate, then the update of y
     EcPlan ep = plan_ec(M, L.K, L.N, L.r, sms);
@@ -302,14 +325,8 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
     return launch_ec(ep, L, x, M, y, hdr, part, tickets, gt, nullptr, nullptr, st, 2);
   }
   if (path == SPEAR_PATH_SEMIFUSED) {
-    LayerView L0 = L;
-    L0.r = 0;
-    L0.agt = nullptr;
-    L0.bpt = nullptr;
-    L0.gate_kind = 0;
-    const bool d2 = M <= 16 && !decode2_unsupported(M, L.K, L.N, L.r, L.gate_kind, L.gate_h);
     auto gemm = [&](float* go, int* mc) {
-      if (d2) return launch_decode2(L0, x, M, y, hdr, tbuf, go, mc, false, st);
+      if (M <= 16) return decode_launch(L0, go, mc, false);
       TcPlan p = plan_tc(M, L.K, L.N, 0, L.group, sms);
       return launch_tc(p, L0, x, M, y, false, hdr, tcflags, gt, go, mc, st);
     };
@@ -384,6 +401,15 @@ const char* spear_status_string(int status) {
 }
 
 int spear_version(void) { return 100; }
+
+int spear_test_inject_timeout(int kernel, long long wait_cycles) {
+  g_last_error.clear();
+  if (kernel < 0 || kernel > 2) return set_error(SPEAR_ERR_INVALID_ARG, "kernel=%d: must be 0, 1 or 2", kernel);
+  if (kernel != 0 && wait_cycles < 1) return set_error(SPEAR_ERR_INVALID_ARG, "wait_cycles must be >= 1");
+  std::lock_guard<std::mutex> lk(g_fault_mu);
+  g_fault = TestFault{kernel, kernel ? wait_cycles : 0};
+  return SPEAR_OK;
+}
 
 size_t spear_w4_packed_bytes(int N, int K) {
   if (N <= 0 || K <= 0 || N % 16 || K % 64) return 0;
@@ -513,7 +539,20 @@ int spear_dispatch_set(int K, int N, int r, int group, int M, int path) {
   if (M < 1) return set_error(SPEAR_ERR_INVALID_ARG, "bad M");
   if (path == SPEAR_PATH_DECODE && M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs M <= 16");
   std::lock_guard<std::mutex> lk(g_dmu);
-  g_table[DKey(K, N, r, group, m_bucket(M))] = DEntry{path, -1.f};
+  g_table[DKey(K, N, r, group, 0, 0, m_bucket(M))] = DEntry{path, -1.f};
+  return SPEAR_OK;
+}
+
+int spear_dispatch_set_layer(const spear_layer* layer, int M, int path, float us) {
+  g_last_error.clear();
+  LayerView L;
+  int rc = check_layer(layer, &L);
+  if (rc) return rc;
+  if (path < SPEAR_PATH_DECODE || path > SPEAR_PATH_SEMIFUSED) return set_error(SPEAR_ERR_INVALID_ARG, "bad path");
+  if (M < 1) return set_error(SPEAR_ERR_INVALID_ARG, "bad M");
+  if (path == SPEAR_PATH_DECODE && M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs M <= 16");
+  std::lock_guard<std::mutex> lk(g_dmu);
+  g_table[dkey(L, M)] = DEntry{path, us >= 0.f ? us : -1.f};
   return SPEAR_OK;
 }
 
@@ -523,7 +562,7 @@ int spear_dispatch_set_time(int K, int N, int r, int group, int M, int path, flo
   const int rc = spear_dispatch_set(K, N, r, group, M, path);
   if (rc) return rc;
   std::lock_guard<std::mutex> lk(g_dmu);
-  g_table[DKey(K, N, r, group, m_bucket(M))].us = us;
+  g_table[DKey(K, N, r, group, 0, 0, m_bucket(M))].us = us;
   return SPEAR_OK;
 }
 
@@ -534,10 +573,10 @@ int spear_dispatch_time_us(const spear_layer* layer, int M, float* us) {
   if (rc) return rc;
   if (M < 1 || !us) return set_error(SPEAR_ERR_INVALID_ARG, "bad M or NULL output");
   std::lock_guard<std::mutex> lk(g_dmu);
-  auto it = g_table.find(DKey(L.K, L.N, L.r, L.group, m_bucket(M)));
+  auto it = g_table.find(dkey(L, M));
   if (it == g_table.end() || it->second.us < 0.f)
-    return set_error(SPEAR_ERR_INVALID_ARG, "no measured time for K=%d N=%d r=%d group=%d at M bucket %d", L.K, L.N,
-                     L.r, L.group, m_bucket(M));
+    return set_error(SPEAR_ERR_INVALID_ARG, "no measured time for K=%d N=%d r=%d group=%d gate=%d at M bucket %d",
+                     L.K, L.N, L.r, L.group, L.r > 0 ? L.gate_kind : 0, m_bucket(M));
   *us = it->second.us;
   return SPEAR_OK;
 }
@@ -571,10 +610,11 @@ int spear_slo_chunk(const spear_layer* const* layers, int n_layers, int decode_t
     float t = step_overhead_us;
     for (int l = 0; l < n_layers; ++l) {
       const LayerView& L = Ls[l];
-      auto it = g_table.find(DKey(L.K, L.N, L.r, L.group, m_bucket(M)));
+      auto it = g_table.find(dkey(L, M));
       if (it == g_table.end() || it->second.us < 0.f)
-        return set_error(SPEAR_ERR_INVALID_ARG, "layer %d (K=%d N=%d r=%d group=%d) has no measured time at M bucket %d",
-                         l, L.K, L.N, L.r, L.group, m_bucket(M));
+        return set_error(SPEAR_ERR_INVALID_ARG,
+                         "layer %d (K=%d N=%d r=%d group=%d gate=%d) has no measured time at M bucket %d", l, L.K,
+                         L.N, L.r, L.group, L.r > 0 ? L.gate_kind : 0, m_bucket(M));
       t += it->second.us;
     }
     if (t <= slo_us && chunk >= best) {
@@ -595,13 +635,17 @@ void spear_dispatch_clear(void) {
 int spear_dispatch_save(const char* path) {
   g_last_error.clear();
   if (!path) return set_error(SPEAR_ERR_INVALID_ARG, "NULL path");
+  int sms = 0;
+  const std::string dev = device_ident(&sms);
   FILE* f = fopen(path, "w");
   if (!f) return set_error(SPEAR_ERR_INVALID_ARG, "cannot open %s for writing", path);
   std::lock_guard<std::mutex> lk(g_dmu);
-  fprintf(f, "# spear dispatch table v2: K N r group M_bucket path time_us (-1 = not measured)\n");
+  fprintf(f, "# spear dispatch table v3 sms=%d device=%s\n", sms, dev.c_str());
+  fprintf(f, "# K N r group gate_kind gate_hidden M_bucket path time_us (-1 = not measured)\n");
   for (const auto& kv : g_table)
-    fprintf(f, "%d %d %d %d %d %d %.3f\n", std::get<0>(kv.first), std::get<1>(kv.first), std::get<2>(kv.first),
-            std::get<3>(kv.first), std::get<4>(kv.first), kv.second.path, kv.second.us);
+    fprintf(f, "%d %d %d %d %d %d %d %d %.3f\n", std::get<0>(kv.first), std::get<1>(kv.first),
+            std::get<2>(kv.first), std::get<3>(kv.first), std::get<4>(kv.first), std::get<5>(kv.first),
+            std::get<6>(kv.first), kv.second.path, kv.second.us);
   fclose(f);
   return SPEAR_OK;
 }
@@ -612,19 +656,54 @@ int spear_dispatch_load(const char* path) {
   FILE* f = fopen(path, "r");
   if (!f) return set_error(SPEAR_ERR_INVALID_ARG, "cannot open %s", path);
   std::map<DKey, DEntry> t;
-  char line[256];
+  char line[512];
   int lineno = 0;
+  bool v3 = false;
   while (fgets(line, sizeof(line), f)) {
     ++lineno;
+    int fsms = 0;
+    char fdev[400];
+    if (sscanf(line, "# spear dispatch table v3 sms=%d device=%399[^\n]", &fsms, fdev) == 2) {
+      // a table measured on another device (name or multiprocessor count) is refused
+      int sms = 0;
+      const std::string dev = device_ident(&sms);
+      if (fsms != sms || dev != fdev) {
+        fclose(f);
+        return set_error(SPEAR_ERR_INVALID_ARG, "%s: table measured on \"%s\" (%d SMs), this device is \"%s\" (%d SMs)",
+                         path, fdev, fsms, dev.c_str(), sms);
+      }
+      v3 = true;
+      continue;
+    }
     if (line[0] == '#' || line[0] == '\n') continue;
-    int K, N, r, g, mb, p;
+    int v[8];
     float us = -1.f;
-    const int n = sscanf(line, "%d %d %d %d %d %d %f", &K, &N, &r, &g, &mb, &p, &us);
-    if ((n != 6 && n != 7) || p < SPEAR_PATH_DECODE || p > SPEAR_PATH_SEMIFUSED || mb < 1) {
+    DKey key;
+    int p = -1;
+    if (v3) {
+      // K N r group gate_kind gate_hidden M_bucket path [time_us]
+      const int n = sscanf(line, "%d %d %d %d %d %d %d %d %f", &v[0], &v[1], &v[2], &v[3], &v[4], &v[5], &v[6],
+                           &v[7], &us);
+      if ((n == 8 || n == 9) && v[6] >= 1 && (v[4] == 0 || v[4] == 1)) {
+        key = DKey(v[0], v[1], v[2], v[3], v[4], v[5], v[6]);
+        p = v[7];
+        if (n == 8) us = -1.f;
+      }
+    } else {
+      // a table without a device line (the earlier format): scalar-gate
+      // entries "K N r group M_bucket path [time_us]"
+      const int n = sscanf(line, "%d %d %d %d %d %d %f", &v[0], &v[1], &v[2], &v[3], &v[4], &v[5], &us);
+      if ((n == 6 || n == 7) && v[4] >= 1) {
+        key = DKey(v[0], v[1], v[2], v[3], 0, 0, v[4]);
+        p = v[5];
+        if (n == 6) us = -1.f;
+      }
+    }
+    if (p < SPEAR_PATH_DECODE || p > SPEAR_PATH_SEMIFUSED) {
       fclose(f);
       return set_error(SPEAR_ERR_INVALID_ARG, "%s:%d: malformed entry", path, lineno);
     }
-    t[DKey(K, N, r, g, mb)] = DEntry{p, us};
+    t[key] = DEntry{p, us};
   }
   fclose(f);
   std::lock_guard<std::mutex> lk(g_dmu);
@@ -696,7 +775,7 @@ int spear_dispatch_tune(const spear_layer* layer, const int* Ms, int nM, const u
     }
     if (result == SPEAR_OK) {
       std::lock_guard<std::mutex> lk(g_dmu);
-      g_table[DKey(L.K, L.N, L.r, L.group, m_bucket(M))] = DEntry{best_path, best < 1e29f ? best : -1.f};
+      g_table[dkey(L, M)] = DEntry{best_path, best < 1e29f ? best : -1.f};
     }
   }
   cudaEventDestroy(e0);

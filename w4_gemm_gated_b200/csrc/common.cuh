@@ -27,7 +27,8 @@ struct WsHeader {
   int gt_obs;     // decode path: CTAs that have read the complete EC projection
   int sf_done;    // semi-fused EC projection launch: CTAs finished
   int sf_count;   // semi-fused EC projection launch: tokens with g < tau
-  int pad0[55];
+  int d3_flag[16];  // decode kernel: EC item e of the current launch published once == d2_epoch + 1
+  int pad0[39];
 };
 static_assert(sizeof(WsHeader) <= 256, "header must fit in 256 bytes");
 constexpr size_t kWsHeaderBytes = 256;
@@ -51,10 +52,10 @@ __device__ __forceinline__ void st_release_gpu(int* p, int v) {
 }
 
 // Spin until *p == want; false (and a status report) if the bound expires.
-__device__ __forceinline__ bool wait_flag_eq(const int* p, int want, WsHeader* h) {
+__device__ __forceinline__ bool wait_flag_eq(const int* p, int want, WsHeader* h, long long limit = kWaitCycles) {
   long long t0 = clock64();
   while (ld_acquire_gpu(p) != want) {
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       report_status(h, SPEAR_ERR_TIMEOUT);
       return false;
     }

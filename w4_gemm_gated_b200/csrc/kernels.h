@@ -16,6 +16,15 @@ int set_cuda_error(const char* what, cudaError_t e);
 // Record a message as the thread's last error; returns `code`.
 int set_error(int code, const char* fmt, ...);
 
+// Failure injection for tests (spear_test_inject_timeout): the kernel whose
+// publication wait is made unsatisfiable (0 none, 1 decode, 2 tensor core),
+// and that wait's bound in SM cycles.
+struct TestFault {
+  int kernel;
+  long long cycles;
+};
+TestFault test_fault();
+
 struct LayerView;
 // Validate a public layer description (same checks as every layer call).
 int validate_layer(const struct spear_layer* layer, LayerView* out);
@@ -60,6 +69,14 @@ const char* decode2_unsupported(int M, int K, int N, int r, int gate_kind, int g
 // bytes of tagged EC projection words the kernel needs in the workspace
 size_t decode2_tt_bytes(int r);
 int launch_decode2(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, WsHeader* hdr, void* tt,
+                   float* gate_out, int* mask_count, bool ec_only, cudaStream_t st);
+
+// ---- decode path without a serial reducer (decode3.cu) ----
+// null if the kernel can run (M, K, N, r, group, gate form), else the reason
+const char* decode3_unsupported(int M, int K, int N, int r, int group, int gate_kind, int gate_h);
+// bytes of published EC rows the kernel needs in the workspace (fits in decode2_tt_bytes(128))
+size_t decode3_tf_bytes();
+int launch_decode3(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, WsHeader* hdr, void* tf,
                    float* gate_out, int* mask_count, bool ec_only, cudaStream_t st);
 
 // ---- standalone EC kernel (ec.cu): y += g * (x.A).B, in place ----

@@ -82,6 +82,8 @@ struct TcArgs {
   const float *gw1, *gb1, *gw2, *gb2;
   float alpha;
   int nst;                // ring stages
+  int tag_skew;           // test injection: projection flags are awaited at epoch + 1 + skew (0 normally)
+  long long pub_wait;     // bound of that wait (SM cycles)
 };
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -220,6 +222,14 @@ __device__ __forceinline__ void dequant_tile(const uint8_t* psrc, uint8_t* bdst,
   }
 }
 
+// Wait, bounded and without reporting, for asynchronous work already issued
+// against this CTA's shared memory or TMEM (before the CTA frees them).
+__device__ __forceinline__ void tc_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitCycles) break;
+}
+
 template <bool GROUP, int BMT>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_kernel(const __grid_constant__ TcArgs a, const __grid_constant__ CUtensorMap tm_x,
@@ -286,6 +296,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
+      int issued = 0;  // stages whose loads went out
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
         const TileInfo ti = tile_info(a, tile);
@@ -338,7 +349,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             if (e == 0) {
               // gated projection of this token block must be published
               for (int qq = 0; qq < 4 * NH && ok; ++qq)
-                ok = wait_flag_eq(&a.mflags[4 * NH * ti.mb + qq], epoch + 1, a.hdr);
+                ok = wait_flag_eq(&a.mflags[4 * NH * ti.mb + qq], epoch + 1 + a.tag_skew, a.hdr, a.pub_wait);
               if (!ok) {
                 *abort_flag = 1;
                 break;
@@ -349,11 +360,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tma_load_2d(smem_u32(xd), &tm_gt, &full[s], e * TC_BK, ti.mb * BMT);
             tma_load_2d(smem_u32(bd), &tm_bpt, &full[s], e * TC_BK, ti.nb * TC_BN);
           }
+          ++issued;
           if (++s == NST) {
             s = 0;
             ph ^= 1;
           }
         }
+      }
+      // Before the CTA exits, no load may still write its shared memory: wait
+      // for the last NST stages issued (a stage has one outstanding phase at
+      // most).  Without an abort they have all been consumed already.
+      for (int j = 0; j < NST && j < issued; ++j) {
+        if (--s < 0) {
+          s = NST - 1;
+          ph ^= 1;
+        }
+        tc_drain(&full[s], ph);
       }
     }
   } else if (warp == 1) {
@@ -363,6 +385,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t ph = 0;
       int buf = 0;
       uint32_t aph[2] = {0, 0};
+      int last_s = -1;      // stage (and its phase) of the last commit
+      uint32_t last_ph = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
         const TileInfo ti = tile_info(a, tile);
@@ -385,6 +409,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               umma(d, ad + 2 * kk, bd + 2 * kk, idesc, (k > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty[s]);
+          last_s = s;
+          last_ph = ph;
           if (++s == NST) {
             s = 0;
             ph ^= 1;
@@ -395,6 +421,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         aph[buf] ^= 1;
         buf = buf + 1 == NBA ? 0 : buf + 1;
       }
+      // the MMAs read shared memory and write TMEM asynchronously: wait for the
+      // last commit (it tracks every earlier MMA) before TMEM is freed
+      if (last_s >= 0) tc_drain(&empty[last_s], last_ph);
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ epilogue
@@ -673,6 +702,9 @@ int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
   a.gb2 = L.gb2;
   a.alpha = L.alpha;
   a.nst = bmt == 256 ? 3 : (a.gate_kind == 1 ? TC_STAGES - 1 : TC_STAGES);
+  const TestFault tf_ = test_fault();
+  a.tag_skew = tf_.kernel == 2 ? 1 : 0;
+  a.pub_wait = tf_.kernel == 2 ? tf_.cycles : kWaitCycles;
   CUtensorMap maps[5];
   memset(maps, 0, sizeof(maps));
   bool ok = tmap_2d_bf16(&maps[0], x, L.K, M, TC_BK, bmt) && tmap_packed_box(&maps[1], L.w, L.K, L.N, 1, TC_BN / 16);

@@ -82,11 +82,14 @@ EXPORTS = {
     "spear_linear_forward_path": (_i, ctypes.POINTER(LayerStruct), _vp, _i, _vp, _vp, _sz, _vp, _vp, _i, _vp),
     "spear_read_status": (_i, _vp, ctypes.POINTER(_i), _vp),
     "spear_linear_forward_decode_noalloc": (_i, ctypes.POINTER(LayerStruct), _vp, _i, _vp, _vp, _vp, _vp),
+    "spear_read_status_noalloc": (_i, ctypes.POINTER(_i), _vp),
+    "spear_test_inject_timeout": (_i, _i, ctypes.c_longlong),
     "spear_dispatch_choice": (_i, ctypes.POINTER(LayerStruct), _i),
     "spear_dispatch_tune": (_i, ctypes.POINTER(LayerStruct), ctypes.POINTER(_i), _i, _vp, _vp, _vp, _sz, _vp, _sz,
                             _i, ctypes.POINTER(_f), _vp),
     "spear_dispatch_set": (_i, _i, _i, _i, _i, _i, _i),
     "spear_dispatch_set_time": (_i, _i, _i, _i, _i, _i, _i, _f),
+    "spear_dispatch_set_layer": (_i, ctypes.POINTER(LayerStruct), _i, _i, _f),
     "spear_dispatch_time_us": (_i, ctypes.POINTER(LayerStruct), _i, ctypes.POINTER(_f)),
     "spear_dispatch_clear": (None,),
     "spear_dispatch_save": (_i, ctypes.c_char_p),
@@ -301,6 +304,20 @@ def read_status(ws: torch.Tensor, stream=None) -> int:
     return v.value
 
 
+def test_inject_timeout(kernel: int, wait_cycles: int = 0) -> None:
+    """Failure injection for tests: make one bounded device wait of the decode
+    (kernel=1) or tensor-core (kernel=2) kernel expire after wait_cycles SM
+    cycles in the launches that follow; kernel=0 turns it off."""
+    _check(F["spear_test_inject_timeout"](kernel, wait_cycles))
+
+
+def read_status_noalloc(stream=None) -> int:
+    """Read and clear the status word of the allocation-free call's array."""
+    v = _i(0)
+    _check(F["spear_read_status_noalloc"](ctypes.byref(v), _stream(stream)))
+    return v.value
+
+
 # --------------------------------------------------------------------------
 # dispatcher
 # --------------------------------------------------------------------------
@@ -328,6 +345,12 @@ def dispatch_set(K: int, N: int, r: int, group: int, M: int, path: int) -> None:
 
 def dispatch_set_time(K: int, N: int, r: int, group: int, M: int, path: int, us: float) -> None:
     _check(F["spear_dispatch_set_time"](K, N, r, group, M, path, us))
+
+
+def dispatch_set_layer(layer, M: int, path: int, us: float = -1.0) -> None:
+    """Set the table entry of this layer's full key (shape, scale kind, gate form)."""
+    st = layer if isinstance(layer, LayerStruct) else layer.struct()
+    _check(F["spear_dispatch_set_layer"](ctypes.byref(st), M, path, us))
 
 
 def dispatch_time_us(layer, M: int) -> float:
