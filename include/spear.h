@@ -178,6 +178,16 @@ typedef struct spear_layer {
   const float* gate_w2;    /* device fp32 r x h row-major                         */
   const float* gate_b2;    /* device fp32 [r]                                     */
   float gate_alpha;        /* alpha of the rank gate                              */
+  /* Optional hint for calls that run layers back to back (a decoder's token
+   * step): the layer the NEXT call on this stream will run, or NULL.  While
+   * this call's decode-path kernel runs, it warms L2 with that layer's packed
+   * weights and EC operands, so the next call's weight loads hit L2 while
+   * DRAM keeps streaming.  A hint only: results are bitwise unchanged, and in
+   * a chain of hinted calls every byte still leaves DRAM once per call.
+   * Read during this call only (its own prefetch_next is ignored); its device
+   * buffers must stay allocated until the next call has run.  The earlier
+   * decode kernels (long or ragged K) and the tensor-core paths ignore it. */
+  const struct spear_layer* prefetch_next;
 } spear_layer;
 
 enum { SPEAR_GATE_SCALAR = 0, SPEAR_GATE_RANK_MLP = 1 };

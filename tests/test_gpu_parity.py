@@ -280,3 +280,21 @@ def test_decode_long_k_rank128_clusters_resident(S, M):
     y_ref, g_ref, _, _ = oracle_ref(L, 0)
     assert_close(y, y_ref)
     assert np.max(np.abs(g.cpu().numpy() - g_ref)) <= GATE_TOL
+
+
+def test_decode_prefetch_hint_leaves_output_unchanged(S, decode_layer):
+    # the prefetch_next hint only warms L2 with the next call's layer: the
+    # output of the hinted call is bitwise the same, at M = 1 and 16
+    L, layer = decode_layer
+    nxt = S.Layer(layer.K, layer.N, 0, layer.r, layer.w_packed.clone(), layer.scales.clone(), layer.AgT.clone(),
+                  layer.BpT.clone(), layer.b_g)
+    for M in (1, 16):
+        x = dev_bf16(L.x[:M])
+        ws = S.make_workspace(layer, M)
+        y0 = S.forward(layer, x, ws, path=S.PATH_DECODE).clone()
+        y1 = S.forward(layer, x, ws, path=S.PATH_DECODE, prefetch_next=nxt).clone()
+        y2 = S.forward(nxt, x, ws, path=S.PATH_DECODE, prefetch_next=layer).clone()
+        torch.cuda.synchronize()
+        assert S.read_status(ws) == S.OK
+        assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+        assert torch.equal(y0.view(torch.int16), y2.view(torch.int16))

@@ -111,6 +111,26 @@ static int check_layer(const spear_layer* l, LayerView* out) {
     out->gb2 = l->gate_b2;
     out->alpha = l->gate_alpha;
   }
+  for (int i = 0; i < 3; ++i) {
+    out->pf[i] = nullptr;
+    out->pf_bytes[i] = 0;
+  }
+  if (const spear_layer* nx = l->prefetch_next) {
+    // the hint's buffers are only prefetched: validate what is read of them
+    if (check_kn(nx->K, nx->N)) return set_error(SPEAR_ERR_INVALID_ARG, "prefetch_next: bad K=%d N=%d", nx->K, nx->N);
+    if (!valid_r(nx->r)) return set_error(SPEAR_ERR_INVALID_ARG, "prefetch_next: bad r=%d", nx->r);
+    if (!nx->w_packed || !aligned16(nx->w_packed) ||
+        (nx->r > 0 && (!nx->AgT || !nx->BpT || !aligned16(nx->AgT) || !aligned16(nx->BpT))))
+      return set_error(SPEAR_ERR_INVALID_ARG, "prefetch_next: NULL or unaligned device pointer");
+    out->pf[0] = nx->w_packed;
+    out->pf_bytes[0] = (size_t)nx->N * nx->K / 2;
+    if (nx->r > 0) {
+      out->pf[1] = nx->AgT;
+      out->pf_bytes[1] = (size_t)(nx->r + 1) * nx->K * 2;
+      out->pf[2] = nx->BpT;
+      out->pf_bytes[2] = (size_t)nx->N * nx->r * 2;
+    }
+  }
   return SPEAR_OK;
 }
 

@@ -43,6 +43,10 @@ struct LayerView {
   int gate_kind, gate_h;
   const float *gw1, *gb1, *gw2, *gb2;  // h x r, h, r x h, r (kind 1)
   float alpha;
+  // the next call's layer, to be warmed in L2 (prefetch_next hint): packed
+  // weights, [A^T ; w_g], B'^T (null / 0 bytes when absent)
+  const void* pf[3];
+  size_t pf_bytes[3];
 };
 
 // ---- decode path (decode.cu) ----

@@ -53,6 +53,7 @@ class LayerStruct(ctypes.Structure):
         ("gate_kind", _i), ("gate_hidden", _i),
         ("gate_w1", _vp), ("gate_b1", _vp), ("gate_w2", _vp), ("gate_b2", _vp),
         ("gate_alpha", _f),
+        ("prefetch_next", _vp),
     ]
 
 
@@ -270,14 +271,19 @@ def make_workspace(layer: Layer, M_max: int, device=None, stream=None) -> torch.
 
 def forward(layer: Layer, x: torch.Tensor, ws: torch.Tensor, y: torch.Tensor | None = None,
             gate_out: torch.Tensor | None = None, mask_count: torch.Tensor | None = None,
-            path: int = PATH_AUTO, stream=None) -> torch.Tensor:
-    """y = x . dequant(W4) + g * ((x . A) . B) for x (M x K bf16) on the device."""
+            path: int = PATH_AUTO, stream=None, prefetch_next: Layer | None = None) -> torch.Tensor:
+    """y = x . dequant(W4) + g * ((x . A) . B) for x (M x K bf16) on the device.
+    prefetch_next: the layer the next call on this stream runs (an L2 warm-up hint)."""
     M, K = x.shape
     if x.dtype != torch.bfloat16:
         raise TypeError("x must be bf16")
     if y is None:
         y = torch.empty((M, layer.N), dtype=torch.bfloat16, device=x.device)
     st = layer.struct()
+    nxt = None
+    if prefetch_next is not None:
+        nxt = prefetch_next.struct()   # kept alive until the call returns
+        st.prefetch_next = ctypes.addressof(nxt)
     _check(F["spear_linear_forward_path"](ctypes.byref(st), _ptr(x), M, _ptr(y), _ptr(ws), ws.numel(),
                                           _ptr(gate_out), _ptr(mask_count), path, _stream(stream)))
     return y
