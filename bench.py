@@ -157,9 +157,9 @@ def time_oracle(target_s: float = 15.0, n_cols: int = 1376):
 # DRAM bytes per decode launch from the ncu captures summarised in profiles/
 # (dram__bytes_read.sum + dram__bytes_write.sum, one launch at M = 1 and at M = 16),
 # valid only while the decode kernel sources are the ones captured.
-DECODE_TRAFFIC = {"sources_sha1": "4b522b75ca9e1e065c18478861b7580446a3dbc5",
-                  "bytes_per_launch": {1: 24639488, 16: 24772608}}
-DECODE_SOURCES = ("w4_gemm_gated_b200/csrc/decode2.cu", "w4_gemm_gated_b200/csrc/common.cuh",
+DECODE_TRAFFIC = {"sources_sha1": "f2b98e5e7fc7764f02807fd11450b3b0ba929d6d",
+                  "bytes_per_launch": {1: 24594688, 16: 24727040}}
+DECODE_SOURCES = ("w4_gemm_gated_b200/csrc/decode3.cu", "w4_gemm_gated_b200/csrc/common.cuh",
                   "w4_gemm_gated_b200/csrc/tma.cuh")
 
 
@@ -207,7 +207,10 @@ def run_reference(args, rank, world):
     value = sum(MS) * args.steps * frac / el
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps / frac,
+        "steps": args.steps, "warmup": args.warmup,
+        # the time of the work actually done: each step computes n_cols of the N output columns
+        "ms_per_step": el * 1e3 / args.steps,
+        "ms_per_step_full_layer_extrapolated": el * 1e3 / args.steps / frac,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": "decode GEMV K=4096 N=11008 r=64, M in {1,4,16} (7B MLP up-projection)",
                    "sample_columns": n_cols},
@@ -230,6 +233,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 32-layer stack (config 4) key")
     ap.add_argument("--profile-case", choices=["decode", "prefill"], default=None,
                     help="run only --steps launches of one kernel on a small case (for ncu captures); "
                          "prints no bench line")
@@ -288,9 +292,12 @@ def main():
 
     def step(i):
         # every launch reads its own weight copy: the copies rotate per launch,
-        # not per step, so no launch finds its weights in L2
+        # not per step, so no launch finds its weights in L2 unless the call
+        # before it warmed them; each call names the next call's layer
+        # (prefetch_next), as a decoder's token step would
         for j, M in enumerate(MS):
-            S.forward(layers[(i * len(MS) + j) % ncopy], xs[M], ws, y=ys[M], stream=stream)
+            c = i * len(MS) + j
+            S.forward(layers[c % ncopy], xs[M], ws, y=ys[M], stream=stream, prefetch_next=layers[(c + 1) % ncopy])
 
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
@@ -356,22 +363,32 @@ def main():
     achieved = tot_bytes / (el_ms * 1e-3 / args.steps) / 1e9
 
     # per-M launch durations (informative): event-free graphs of one M only
-    def per_launch_us(lays, M):
+    def per_launch_stats(lays, M, reps=12):
+        """Back-to-back launches of one M (a graph of 3 x copies launches, hinted):
+        the mean launch time of each replay; median, p10 and p90 over replays."""
+        n = 3 * ncopy
         gm = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gm, stream=stream):
-            for i in range(3 * ncopy):
-                S.forward(lays[i % ncopy], xs[M], ws, y=ys[M], stream=stream)
+            for i in range(n):
+                S.forward(lays[i % ncopy], xs[M], ws, y=ys[M], stream=stream, prefetch_next=lays[(i + 1) % ncopy])
+        vals = []
         with torch.cuda.stream(stream):
             gm.replay()
-            m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            m0.record(stream)
-            for _ in range(4):
+            for _ in range(reps):
+                m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                m0.record(stream)
                 gm.replay()
-            m1.record(stream)
-        m1.synchronize()
-        return m0.elapsed_time(m1) * 1e3 / (4 * 3 * ncopy)
+                m1.record(stream)
+                m1.synchronize()
+                vals.append(m0.elapsed_time(m1) * 1e3 / n)
+        return {"median": float(np.median(vals)), "p10": float(np.percentile(vals, 10)),
+                "p90": float(np.percentile(vals, 90))}
 
-    mean_us = {M: per_launch_us(layers, M) for M in MS}
+    def per_launch_us(lays, M):
+        return per_launch_stats(lays, M)["median"]
+
+    launch_stats = {M: per_launch_stats(layers, M) for M in MS}
+    mean_us = {M: launch_stats[M]["median"] for M in MS}
     # the pages' per-rank gate gamma(t) (bottleneck h = 16) on the same layers
     rng = np.random.default_rng(7)
     rg = [torch.from_numpy(v.astype(np.float32)).to(dev) for v in
@@ -393,7 +410,8 @@ def main():
         def e2e_step(i):
             for j, M in enumerate(MS):
                 dx[M].copy_(hx[M], non_blocking=True)
-                S.forward(layers[(i * len(MS) + j) % ncopy], dx[M], ws, y=ys[M], stream=stream)
+                c = i * len(MS) + j
+                S.forward(layers[c % ncopy], dx[M], ws, y=ys[M], stream=stream, prefetch_next=layers[(c + 1) % ncopy])
                 hy[M].copy_(ys[M], non_blocking=True)
         for i in range(3):
             e2e_step(i)
@@ -410,23 +428,21 @@ def main():
 
     # ---- EC overhead: same kernel with the EC disabled ----
     plain = [S.Layer(K_, N_, 0, 0, lay.w_packed, lay.scales, None, None, 0.0) for lay in layers]
-    gp = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gp, stream=stream):
-        for i in range(3 * ncopy):
-            S.forward(plain[i % ncopy], xs[16], ws, y=ys[16], stream=stream)
-    with torch.cuda.stream(stream):
-        gp.replay()
-        n0, n1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n0.record(stream)
-        for _ in range(4):
-            gp.replay()
-        n1.record(stream)
-    n1.synchronize()
-    noec_us = n0.elapsed_time(n1) * 1e3 / (4 * 3 * ncopy)
+    noec_us = per_launch_us(plain, 16)
+    noec_us_m1 = per_launch_us(plain, 1)
 
     prefill = None
     if not args.no_prefill and rank == 0:
         prefill = bench_prefill(S, synth, dev, stream, bf16, tc_peak)
+    stack = None
+    if not args.no_stack and rank == 0:
+        try:
+            stack = stack_measure(S, synth, 5)
+            stack["roofline"] = {"bound": "tensor", "achieved": stack["linears_tflops"], "peak": tc_sust,
+                                 "unit": "TFLOP/s", "frac": stack["linears_tflops"] / tc_sust,
+                                 "peak_source": f"{peak_src} bf16_tflops_sustained (a long step)"}
+        except Exception as e:  # report, do not hide the decode result
+            stack = {"error": f"{type(e).__name__}: {e}"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -449,18 +465,25 @@ def main():
                    "tokens_per_step": tokens_per_step, "parallelism": f"replicas x{world}",
                    "l2": f"cold: {ncopy} weight copies rotating per launch ({ncopy * layer_bytes / 1e6:.0f} MB > 2x L2)",
                    "timing": f"CUDA-graph replay of {chunk}-step chunks (launches overlap through programmatic "
-                             f"dependent launch), events on the launching stream"},
+                             f"dependent launch), events on the launching stream",
+                   "prefetch_hint": "each call names the next call's layer (prefetch_next): its kernel warms L2 "
+                                    "with that layer's weights; DRAM bytes per step unchanged"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": decode_traffic_per_step(),
                      "traffic_unit": "DRAM bytes per step (3 launches), ncu capture in profiles/",
                      "kernel": "decode_kernel (fused W4 GEMV + gated EC)",
                      "per_launch_us": mean_us,
+                     "per_launch_us_p10_p50_p90": {M: [launch_stats[M]["p10"], launch_stats[M]["median"],
+                                                       launch_stats[M]["p90"]] for M in MS},
                      "achieved_from": "algorithmic bytes of a step / timed step time (3 decode launches)",
-                     "per_launch_timing": "event-free graphs of 3 x copies launches of one M, back to back",
+                     "per_launch_timing": "event-free graphs of 3 x copies launches of one M, back to back; "
+                                          "p10/p50/p90 over 12 replays of the mean launch time",
                      "algorithmic_bytes": {M: alg_bytes(M, K_, N_, R_) for M in MS},
                      "peak_source": f"{peak_src} hbm_gbs"},
         "ec_overhead": {"m16_with_ec_us": mean_us[16], "m16_ec_disabled_us": noec_us,
-                        "overhead": mean_us[16] / noec_us - 1.0},
+                        "overhead": mean_us[16] / noec_us - 1.0,
+                        "m1_with_ec_us": mean_us[1], "m1_ec_disabled_us": noec_us_m1,
+                        "overhead_m1": mean_us[1] / noec_us_m1 - 1.0},
         "rank_gate": {"per_launch_us": rank_us, "hidden": 16,
                       "vs_scalar_gate": {M: rank_us[M] / mean_us[M] - 1.0 for M in rank_us},
                       "form": "y = xW + alpha (t * sigmoid(W2 relu(W1 t + b1) + b2)) B, t = xA"},
@@ -473,6 +496,8 @@ def main():
     }
     if prefill is not None:
         line["prefill"] = prefill
+    if stack is not None:
+        line["stack"] = stack
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -593,14 +618,18 @@ def stack_glue(S, layers, x, ws, eps=1e-6, n_layers=32):
 
 
 def run_stack(args):
+    from w4_gemm_gated_b200 import spear as S
+    from w4_gemm_gated_b200 import synth
+    print(json.dumps(stack_measure(S, synth, max(1, min(args.steps, 5)))))
+
+
+def stack_measure(S, synth, reps):
     """Config 4: 32 decoder layers x 7 per-channel W4 linears, ECs (r=64) on all
     linears of layers 0, 1, 30, 31, M=256 tokens pushed through all 224 linears.
     Weights are drawn on the device (seeded per projection) and quantised and
     packed by the library.  Reports the time of the linears alone and of the
-    whole stack with the glue."""
+    whole stack with the glue (mean of `reps` passes, with p10/p90)."""
     import torch
-    from w4_gemm_gated_b200 import spear as S
-    from w4_gemm_gated_b200 import synth
 
     M, R = 256, 64
     dev = torch.device("cuda")
@@ -636,40 +665,48 @@ def run_stack(args):
             for lay in row:
                 S.forward(lay, xs[lay.K], ws)
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = max(1, min(args.steps, 5))
-    a.record(stream)
+    lin = []
     for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
         for row in layers:
             for lay in row:
                 S.forward(lay, xs[lay.K], ws)
-    b.record(stream)
-    b.synchronize()
-    lin_ms = a.elapsed_time(b) / reps
+        b.record(stream)
+        b.synchronize()
+        lin.append(a.elapsed_time(b))
+    lin_ms = float(np.mean(lin))
 
     # the whole stack with the glue
     for _ in range(2):
         out = stack_glue(S, layers, x0, ws)
     torch.cuda.synchronize()
-    a.record(stream)
+    full = []
     for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
         out = stack_glue(S, layers, x0, ws)
-    b.record(stream)
-    b.synchronize()
-    e2e_ms = a.elapsed_time(b) / reps
+        b.record(stream)
+        b.synchronize()
+        full.append(a.elapsed_time(b))
+    e2e_ms = float(np.mean(full))
     assert S.read_status(ws) == S.OK
     finite = bool(torch.isfinite(out.float()).all().item())
     flops = sum(2.0 * M * K * N for (K, N) in STACK_SHAPES) * 32 + \
         len(STACK_EC_LAYERS) * sum(2.0 * M * K * (R + 1) + 2.0 * M * R * N for (K, N) in STACK_SHAPES)
-    print(json.dumps({
+    del layers, ws
+    torch.cuda.empty_cache()
+    return {
         "stack": "32 decoder layers x 7 W4 linears, ECs r=64 on layers 0,1,30,31", "M": M,
         "linears_ms": lin_ms, "stack_ms": e2e_ms, "tokens_per_s": M / (e2e_ms * 1e-3),
+        "linears_ms_p10_p90": [float(np.percentile(lin, 10)), float(np.percentile(lin, 90))],
+        "stack_ms_p10_p90": [float(np.percentile(full, 10)), float(np.percentile(full, 90))],
         "linears_tflops": flops / (lin_ms * 1e-3) / 1e12,
         "packed_weight_bytes": packed_bytes, "ec_params": ec_params,
         "ec_params_fraction_of_packed_bytes": ec_params / packed_bytes,
         "ec_bytes_fraction_of_packed_bytes": 2 * ec_params / packed_bytes,
         "output_finite": finite, "prep_seconds": round(prep_s, 1),
-        "timing": f"mean of {reps} passes, weights 3.24 GB (no L2 reuse across passes)"}))
+        "timing": f"mean of {reps} passes, weights 3.24 GB (no L2 reuse across passes)"}
 
 
 def run_profile_case(args):
@@ -734,6 +771,7 @@ def bench_prefill(S, synth, dev, stream, bf16, tc_peak):
                     if i >= 3:
                         ts.append(a.elapsed_time(b) * 1e3)
             res[name] = float(np.median(ts))
+            res[name + "_p10_p90"] = [float(np.percentile(ts, 10)), float(np.percentile(ts, 90))]
         if S.read_status(ws, stream=stream) != S.OK:
             return {"error": "device status not OK"}
         fl = alg_flops(2048, 4096, 4096, 64)
@@ -745,6 +783,7 @@ def bench_prefill(S, synth, dev, stream, bf16, tc_peak):
                 "roofline": {"bound": "tensor", "achieved": tf, "peak": tc_peak, "unit": "TFLOP/s",
                              "frac": tf / tc_peak},
                 "ec_overhead": res["fused"] / res["ec_disabled"] - 1.0,
+                "fused_us_p10_p90": res["fused_p10_p90"], "ec_disabled_us_p10_p90": res["ec_disabled_p10_p90"],
                 "timing": "median of 10 single launches, L2 flushed (256 MB write) before each"}
     except Exception as e:  # report, do not hide the decode result
         return {"error": f"{type(e).__name__}: {e}"}

@@ -102,8 +102,8 @@ __host__ __device__ __forceinline__ D3Smem d3_smem(int MT, int ubytes, int own_c
   off += gate_kind == 1 ? d3_up(MT * (32 + r) * 4, 16) : 0;
   s.stage = off;  // per warp [MT tokens][16 channels] bf16
   off += D3_NW * MT * 32;
-  s.bars = off;  // unit barriers, epilogue operands, fetched t
-  off += (D3_MAXU + 2) * 8;
+  s.bars = off;  // unit barriers, partials complete, epilogue operands, fetched t, gt ready
+  off += (2 * D3_MAXU + 3) * 8;
   s.total = off + 1024;  // base alignment slack
   return s;
 }
@@ -534,8 +534,12 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
   float* ts = reinterpret_cast<float*>(sm + SL.ts);
   float* gpart = reinterpret_cast<float*>(sm + SL.gpart);
   uint64_t* ubar = reinterpret_cast<uint64_t*>(sm + SL.bars);
-  uint64_t* epibar = ubar + D3_MAXU;
+  uint64_t* pbar = ubar + D3_MAXU;  // every warp's partial of unit u written (16 arrivals)
+  uint64_t* epibar = pbar + D3_MAXU;
   uint64_t* tsbar = epibar + 1;
+  uint64_t* gtbar = tsbar + 1;      // gt built (scalar gate)
+  __nv_bfloat16* gts = reinterpret_cast<__nv_bfloat16*>(sm + SL.gts);
+  float* gv = reinterpret_cast<float*>(sm + SL.gv);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rho = lane >> 2, c = lane & 3;
@@ -549,10 +553,14 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
   auto ubase = [&](int u) { return units + d3_unit_off(u, n_ecu, ecu, a.wunit); };
 
   if (warp == 0) {
-    for (int u = lane; u < U; u += 32) mbar_init(&ubar[u], 1);
+    for (int u = lane; u < U; u += 32) {
+      mbar_init(&ubar[u], 1);
+      mbar_init(&pbar[u], D3_NW);
+    }
     if (lane == 0) {
       mbar_init(epibar, 1);
       mbar_init(tsbar, 32);
+      mbar_init(gtbar, 1);
       s_abort = 0;
       s_eccnt = 0;
       s_fetched = 0;
@@ -622,14 +630,14 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // x, y and the workspace may belong to the previous kernel in the stream
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int tag = *reinterpret_cast<volatile int*>(&a.hdr->d2_epoch) + 1;
   if (!has_ec && blockIdx.x == 0 && warp == 1) {
     if (a.gate_out && lane < a.M) a.gate_out[lane] = 0.f;
     if (a.mask_count && lane == 0) *a.mask_count = a.M;
   }
 
   // activations of this warp's k slice as B fragments: word i of xf[t][nt]
-  // = x[nt*8 + rho][64 (w CH + t) + 16c + 2i .. + 1]
+  // = x[nt*8 + rho][64 (w CH + t) + 16c + 2i .. + 1]; requested before the
+  // launch tag, whose read then overlaps them
   uint32_t xf[CH][NT][8];
 #pragma unroll
   for (int t = 0; t < CH; ++t)
@@ -645,6 +653,10 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
       xf[t][nt][0] = v0.x; xf[t][nt][1] = v0.y; xf[t][nt][2] = v0.z; xf[t][nt][3] = v0.w;
       xf[t][nt][4] = v1.x; xf[t][nt][5] = v1.y; xf[t][nt][6] = v1.z; xf[t][nt][7] = v1.w;
     }
+  const int tag = *reinterpret_cast<volatile int*>(&a.hdr->d2_epoch) + 1;
+  // every warp has its tag before any warp of this CTA can count the CTA as
+  // done with this launch's rows (which lets the epoch advance)
+  __syncthreads();
   // per-channel codes enter the MMAs as 136 + q: remove 136 * sum(x) of the
   // slice per token (accumulator columns 2c and 2c + 1 of each n8 tile)
   float xsA[NT], xsB[NT];
@@ -760,6 +772,8 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
       for (int nt = 0; nt < NT; ++nt)
         *reinterpret_cast<float4*>(base + warp * CH * 512 + nt * 512 + lane * 16) =
             make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pbar[u]);
       if (fetcher && !s_fetched && d3_flags_ready(a, tag)) {
         d3_fetch_t<MT>(a, ts, tsbar, lane);
         if (lane == 0) s_fetched = 1;
@@ -795,18 +809,58 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
       __syncwarp();
     }
   }
-  if (fetcher && s_fetched) __all_sync(FULL, d3_wait(tsbar, 0, abortp, a.hdr));
+  if (fetcher && s_fetched) ok = __all_sync(FULL, d3_wait(tsbar, 0, abortp, a.hdr));
+  if (fetcher && ok && a.gate_kind == 0) {
+    // scalar gate, by this warp alone: g = sigmoid(logit + b_g) and
+    // gt = bf16(g t) for the live tokens (zero rows for the padded ones);
+    // the strip warps wait on gtbar, not on the whole CTA
+    const int gs = a.r + 8, half = a.r / 2;
+    if (lane < MT) gv[lane] = lane < a.M ? sigmoidf_(ts[MT * a.r + lane] + a.b_g) : 0.f;
+    __syncwarp();
+    for (int idx = lane; idx < MT * half; idx += 32) {
+      const int m = idx / half, j = 2 * (idx - m * half);
+      const float g = gv[m];
+      *reinterpret_cast<uint32_t*>(gts + m * gs + j) =
+          m < a.M ? pack_bf16x2(g * ts[m * a.r + j], g * ts[m * a.r + j + 1]) : 0u;
+    }
+    if (blockIdx.x == 0) {
+      const bool valid = lane < a.M;
+      const float g = lane < MT ? gv[lane] : 0.f;
+      if (a.gate_out && valid) a.gate_out[lane] = g;
+      const unsigned below = __ballot_sync(FULL, valid && g < a.tau);
+      if (a.mask_count && lane == 0) *a.mask_count = __popc(below);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(gtbar);
+  }
 
   // ------------------------------------------------------------------ end phase
-  __syncthreads();
-  // Read once by every thread between two barriers: nothing writes the flag
-  // before the gate block's last barrier, so the branch below is uniform.
-  const bool live = !*abortp;
-  if (needs_t && live) d3_build_gate<MT>(a, sm);
+  bool live = true;
+  if (has_ec && a.gate_kind == 1) {
+    // the pages' per-rank gate: built by the whole CTA (its MLP is the bulk of it)
+    __syncthreads();
+    // Read once by every thread between two barriers: nothing writes the flag
+    // before the gate block's last barrier, so the branch below is uniform.
+    live = !*abortp;
+    if (needs_t && live) d3_build_gate<MT>(a, sm);
+  }
   if (live) {
-    bool eok = __all_sync(FULL, d3_wait(epibar, 0, abortp, a.hdr));
-    for (int j = warp; j < n_w && eok; j += D3_NW)
-      d3_finish_strip<MT, GROUP>(a, sm, j, w_lo + j, ubase(n_ecu + j), CH, lane, warp);
+    // strip j by warp j % 16, as soon as its 16 partials (and gt) are ready
+    bool eok = n_w > warp ? __all_sync(FULL, d3_wait(epibar, 0, abortp, a.hdr)) : false;
+    for (int j = warp; j < n_w && eok; j += D3_NW) {
+      if (!a.ec_only) eok = __all_sync(FULL, d3_wait(&pbar[n_ecu + j], 0, abortp, a.hdr));
+      if (eok && has_ec && a.gate_kind == 0) eok = __all_sync(FULL, d3_wait(gtbar, 0, abortp, a.hdr));
+      if (eok) d3_finish_strip<MT, GROUP>(a, sm, j, w_lo + j, ubase(n_ecu + j), CH, lane, warp);
+    }
+  }
+  // every CTA reads this launch's rows at most once; the last one to be done
+  // with them advances the epoch (CTAs that never read them count as well)
+  const bool t_done = needs_t ? (fetcher && ok && s_fetched) : (warp == 0);
+  if (has_ec && t_done && lane == 0 && !*abortp) {
+    if (atomicAdd(&a.hdr->gt_obs, 1) == a.G - 1) {
+      a.hdr->gt_obs = 0;
+      a.hdr->d2_epoch = tag;
+    }
   }
   if (warp == 0) {
     // no copy may still write into this CTA's shared memory when it exits
@@ -814,13 +868,6 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
     for (int u = 0; u < U; ++u) d3_drain(&ubar[u], 0);
     d3_drain(epibar, 0);
     if (s_fetched) d3_drain(tsbar, 0);
-  }
-  if (has_ec && threadIdx.x == 0 && live && !*abortp) {
-    // every CTA has read this launch's rows; the last one advances the epoch
-    if (atomicAdd(&a.hdr->gt_obs, 1) == a.G - 1) {
-      a.hdr->gt_obs = 0;
-      a.hdr->d2_epoch = tag;
-    }
   }
 }
 
