@@ -102,4 +102,6 @@ def test_two_layer_pipeline_against_oracle(S):
     ref = _oracle_stack(O.bf16_to_f64(x_bits), mats)
     got = _f64(out)
     assert np.all(np.isfinite(got))
-    assert np.max(np.abs(got - ref)) <= 2e-2 * np.max(np.abs(ref))
+    # the oracle pipeline rounds to bf16 at the same points as the device glue,
+    # so the per-linear bound holds across the 14 linears as well
+    assert np.max(np.abs(got - ref)) <= 1e-2 * np.max(np.abs(ref))

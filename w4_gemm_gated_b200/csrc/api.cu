@@ -141,7 +141,7 @@ int device_sm_count() { return sm_count(); }
 // workspace layout
 // ---------------------------------------------------------------------------
 struct WsLayout {
-  size_t hdr, tickets, tcflags, t, gt, part, total;
+  size_t hdr, tickets, tcflags, kflags, t, gt, part, kpart, total;
   int n_flags;
 };
 
@@ -153,6 +153,7 @@ static size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 // scratch after them (gated projection, K-split partials) grows with M.
 static constexpr int kMaxM = 65536;
 static constexpr int kFlagCap = kMaxM / 16 + 64;  // 16-token blocks (+ slack)
+static constexpr int kKFlagCap = 4 * 1024;         // K-part flags: 4 per (tile, part), tiles x parts <= SMs
 
 static WsLayout ws_layout_uncached(const LayerView& L, int M_max) {
   WsLayout w = {};
@@ -165,6 +166,8 @@ static WsLayout ws_layout_uncached(const LayerView& L, int M_max) {
   off = up256(off + sizeof(int) * kFlagCap);
   w.tcflags = off;
   off = up256(off + sizeof(int) * 4 * kFlagCap);
+  w.kflags = off;
+  off = up256(off + sizeof(int) * kKFlagCap);
   w.t = off;
   off = up256(off + sizeof(float) * std::max<size_t>(16 * (size_t)RT, decode2_tt_bytes(128) / sizeof(float)));
   w.gt = off;
@@ -179,6 +182,10 @@ static WsLayout ws_layout_uncached(const LayerView& L, int M_max) {
     }
   }
   off = up256(off + sizeof(float) * part_floats);
+  // K-part partial accumulators of the tensor-core tiles (M > 16): tiles x
+  // parts <= SMs, each 128 tokens x 256 channels fp32
+  w.kpart = off;
+  off = up256(off + (M_max > 16 ? (size_t)sm_count() * 128 * 256 * sizeof(float) : 0));
   w.total = off;
   return w;
 }
@@ -294,6 +301,8 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + wl.hdr);
   int* tickets = reinterpret_cast<int*>(ws + wl.tickets);
   int* tcflags = reinterpret_cast<int*>(ws + wl.tcflags);
+  int* kflags = reinterpret_cast<int*>(ws + wl.kflags);
+  float* kpart = wl.total > wl.kpart ? reinterpret_cast<float*>(ws + wl.kpart) : nullptr;
   float* tbuf = reinterpret_cast<float*>(ws + wl.t);
   __nv_bfloat16* gt = reinterpret_cast<__nv_bfloat16*>(ws + wl.gt);
   float* part = reinterpret_cast<float*>(ws + wl.part);
@@ -335,7 +344,7 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
       return decode_launch(L, gate_out, mask_count, true);
     }
     TcPlan p = plan_tc(M, L.K, L.N, 0, L.group, sms);
-    rc = launch_tc(p, L0, x, M, y, false, hdr, tcflags, gt, L.r > 0 ? nullptr : gate_out,
+    rc = launch_tc(p, L0, x, M, y, false, hdr, tcflags, kflags, kpart, gt, L.r > 0 ? nullptr : gate_out,
                    L.r > 0 ? nullptr : mask_count, st);
     if (rc || L.r == 0) return rc;
     // the separate EC kernel: projection and gate, then the update of y
@@ -348,7 +357,7 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
     auto gemm = [&](float* go, int* mc) {
       if (M <= 16) return decode_launch(L0, go, mc, false);
       TcPlan p = plan_tc(M, L.K, L.N, 0, L.group, sms);
-      return launch_tc(p, L0, x, M, y, false, hdr, tcflags, gt, go, mc, st);
+      return launch_tc(p, L0, x, M, y, false, hdr, tcflags, kflags, kpart, gt, go, mc, st);
     };
     if (L.r == 0) return gemm(gate_out, mask_count);
     const EcPlan ep = plan_ec(M, L.K, L.N, L.r, sms);
@@ -371,7 +380,7 @@ static int run_path(const LayerView& L, const __nv_bfloat16* x, int M, __nv_bflo
   }
   if (path == SPEAR_PATH_FUSED) {
     TcPlan p = plan_tc(M, L.K, L.N, L.r, L.group, sms);
-    return launch_tc(p, L, x, M, y, L.r > 0, hdr, tcflags, gt, gate_out, mask_count, st);
+    return launch_tc(p, L, x, M, y, L.r > 0, hdr, tcflags, kflags, kpart, gt, gate_out, mask_count, st);
   }
   return set_error(SPEAR_ERR_INVALID_ARG, "unknown path %d", path);
 }

@@ -51,6 +51,31 @@ __device__ __forceinline__ void st_release_gpu(int* p, int v) {
   asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Spin until the n flags f[0..n) all equal want, their loads in flight
+// together (one round trip per poll), then an acquire fence; false (and a
+// status report) if the bound expires.
+__device__ __forceinline__ bool wait_flags_eq(const int* f, int n, int want, WsHeader* h, long long limit) {
+  const long long t0 = clock64();
+  for (;;) {
+    int v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (i < n) asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v[i]) : "l"(f + i) : "memory");
+    bool all = true;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (i < n) all = all && v[i] == want;
+    if (all) break;
+    if (clock64() - t0 > limit) {
+      report_status(h, SPEAR_ERR_TIMEOUT);
+      return false;
+    }
+    __nanosleep(32);
+  }
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+  return true;
+}
+
 // Spin until *p == want; false (and a status report) if the bound expires.
 __device__ __forceinline__ bool wait_flag_eq(const int* p, int want, WsHeader* h, long long limit = kWaitCycles) {
   long long t0 = clock64();

@@ -105,7 +105,8 @@ struct TcPlan {
 };
 TcPlan plan_tc(int M, int K, int N, int r, int group, int sm_count);
 int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, bool with_ec,
-              WsHeader* hdr, int* mflags, __nv_bfloat16* gt, float* gate_out, int* mask_count, cudaStream_t st);
+              WsHeader* hdr, int* mflags, int* kflags, float* kpart, __nv_bfloat16* gt, float* gate_out,
+              int* mask_count, cudaStream_t st);
 
 // ---- packing kernels (pack.cu) ----
 int launch_quantize(const float* W, int K, int N, int group, int8_t* q, __half* s, cudaStream_t st);

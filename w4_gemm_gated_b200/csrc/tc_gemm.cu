@@ -84,6 +84,9 @@ struct TcArgs {
   int nst;                // ring stages
   int tag_skew;           // test injection: projection flags are awaited at epoch + 1 + skew (0 normally)
   long long pub_wait;     // bound of that wait (SM cycles)
+  int S;                  // K parts per tile (1: none); CTA b takes part b % S of tiles b / S, + grid / S, ...
+  float* kpart;           // [tiles * S][4 warps][64][32 lanes][4] fp32 partial accumulators (S > 1)
+  int* kflags;            // [tiles * S][4 * NH]: epoch + 1 once an epilogue warp's partial rows are out
 };
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -132,6 +135,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
   asm volatile(
@@ -149,26 +164,30 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 // schedule shared by all roles
 // ---------------------------------------------------------------------------
 struct TileInfo {
-  int kind;  // 0 = projection tile, 1 = output tile
+  int kind;    // 0 = projection tile, 1 = output tile
   int mb, nb;
-  int steps;  // k-steps of this tile
+  int k0, nk;  // this CTA's K part of the tile: k-steps k0 .. k0 + nk - 1
+  int steps;   // k-steps of this tile in this CTA (its K part, then the EC steps in the last part)
 };
 
 __device__ __forceinline__ TileInfo tile_info(const TcArgs& a, int tile) {
   TileInfo t;
   const int KT = a.K / TC_BK;
   const int nproj = a.with_ec ? a.Mb : 0;
+  const int part = (int)(blockIdx.x % (unsigned)a.S);
+  t.nk = KT / a.S;
+  t.k0 = part * t.nk;
   if (tile < nproj) {
     t.kind = 0;
     t.mb = tile;
     t.nb = 0;
-    t.steps = KT;
+    t.steps = t.nk;
   } else {
     const int i = tile - nproj;
     t.kind = 1;
     t.mb = i / a.Nb;
     t.nb = i % a.Nb;
-    t.steps = KT + (a.with_ec ? a.ec_steps : 0);
+    t.steps = t.nk + (a.with_ec && part == a.S - 1 ? a.ec_steps : 0);
   }
   return t;
 }
@@ -261,6 +280,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int epoch = *reinterpret_cast<volatile int*>(&a.hdr->epoch);
   const int ntiles = (a.with_ec ? a.Mb : 0) + a.Mb * a.Nb;
+  // tiles of this CTA: groups of S consecutive CTAs share each tile's K parts
+  const int t_first = (int)blockIdx.x / a.S, t_step = (int)gridDim.x / a.S;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -298,9 +319,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t ph = 0;
       int issued = 0;  // stages whose loads went out
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int tile = t_first; tile < ntiles && ok; tile += t_step) {
         const TileInfo ti = tile_info(a, tile);
-        const int KT = a.K / TC_BK;
         for (int k = 0; k < ti.steps && ok; ++k) {
           ok = mbar_wait(&empty[s], ph ^ 1, abort_flag, a.hdr);
           if (!ok) break;
@@ -309,56 +329,57 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           uint8_t* pd = ps + s * TC_P_BYTES;
           if (ti.kind == 0) {
             mbar_arrive_tx(&full[s], XB + a.NE * 128);
-            tma_load_2d(smem_u32(xd), &tm_x, &full[s], k * TC_BK, ti.mb * BMT);
-            tma_load_2d(smem_u32(bd), &tm_agt, &full[s], k * TC_BK, 0);
-          } else if (k < KT) {
+            tma_load_2d(smem_u32(xd), &tm_x, &full[s], (ti.k0 + k) * TC_BK, ti.mb * BMT);
+            tma_load_2d(smem_u32(bd), &tm_agt, &full[s], (ti.k0 + k) * TC_BK, 0);
+          } else if (k < ti.nk) {
+            const int kg = ti.k0 + k;
             // warm L2 a few k-steps ahead so the shallow shared-memory ring
             // does not see the full HBM latency on every stage
-            if (k + TC_PREFETCH < KT) {
-              tma_prefetch_2d(&tm_x, (k + TC_PREFETCH) * TC_BK, ti.mb * BMT);
-              tma_prefetch_3d(&tm_w, 0, k + TC_PREFETCH, ti.nb * (TC_BN / 16));
+            if (k + TC_PREFETCH < ti.nk) {
+              tma_prefetch_2d(&tm_x, (kg + TC_PREFETCH) * TC_BK, ti.mb * BMT);
+              tma_prefetch_3d(&tm_w, 0, kg + TC_PREFETCH, ti.nb * (TC_BN / 16));
             } else {
               // the tile's tail: warm its EC operands (L2 is coherent, so gt may
               // be warmed before the projection is published) and the first
               // k-steps of this CTA's next tile
-              const int j = k + TC_PREFETCH - KT;
-              if (j == 0 && a.with_ec)
+              const int j = k + TC_PREFETCH - ti.nk;
+              if (j == 0 && ti.steps > ti.nk)
                 for (int e = 0; e < a.ec_steps; ++e) {
                   tma_prefetch_2d(&tm_bpt, e * TC_BK, ti.nb * TC_BN);
                   tma_prefetch_2d(&tm_gt, e * TC_BK, ti.mb * BMT);
                 }
-              const int nt = tile + (int)gridDim.x;
+              const int nt = tile + t_step;
               if (nt < ntiles) {
                 const TileInfo tn = tile_info(a, nt);
-                if (tn.kind == 1 && j < KT) {
-                  tma_prefetch_2d(&tm_x, j * TC_BK, tn.mb * BMT);
-                  tma_prefetch_3d(&tm_w, 0, j, tn.nb * (TC_BN / 16));
+                if (tn.kind == 1 && j < tn.nk) {
+                  tma_prefetch_2d(&tm_x, (tn.k0 + j) * TC_BK, tn.mb * BMT);
+                  tma_prefetch_3d(&tm_w, 0, tn.k0 + j, tn.nb * (TC_BN / 16));
                 }
               }
             }
             if (k == 0)
-              for (int pk = 1; pk < TC_PREFETCH && pk < KT; ++pk) {
-                tma_prefetch_2d(&tm_x, pk * TC_BK, ti.mb * BMT);
-                tma_prefetch_3d(&tm_w, 0, pk, ti.nb * (TC_BN / 16));
+              for (int pk = 1; pk < TC_PREFETCH && pk < ti.nk; ++pk) {
+                tma_prefetch_2d(&tm_x, (ti.k0 + pk) * TC_BK, ti.mb * BMT);
+                tma_prefetch_3d(&tm_w, 0, ti.k0 + pk, ti.nb * (TC_BN / 16));
               }
             mbar_arrive_tx(&full[s], XB + TC_P_BYTES);
-            tma_load_2d(smem_u32(xd), &tm_x, &full[s], k * TC_BK, ti.mb * BMT);
-            tma_load_3d(smem_u32(pd), &tm_w, &full[s], 0, k, ti.nb * (TC_BN / 16));
+            tma_load_2d(smem_u32(xd), &tm_x, &full[s], kg * TC_BK, ti.mb * BMT);
+            tma_load_3d(smem_u32(pd), &tm_w, &full[s], 0, kg, ti.nb * (TC_BN / 16));
           } else {
-            const int e = k - KT;
+            const int e = k - ti.nk;
+            // B' does not depend on the projection: its load goes out first
+            mbar_arrive_tx(&full[s], XB + TC_B_BYTES);
+            tma_load_2d(smem_u32(bd), &tm_bpt, &full[s], e * TC_BK, ti.nb * TC_BN);
             if (e == 0) {
-              // gated projection of this token block must be published
-              for (int qq = 0; qq < 4 * NH && ok; ++qq)
-                ok = wait_flag_eq(&a.mflags[4 * NH * ti.mb + qq], epoch + 1 + a.tag_skew, a.hdr, a.pub_wait);
-              if (!ok) {
-                *abort_flag = 1;
-                break;
-              }
+              // gated projection of this token block must be published (all
+              // its flags polled together)
+              ok = wait_flags_eq(&a.mflags[4 * NH * ti.mb], 4 * NH, epoch + 1 + a.tag_skew, a.hdr, a.pub_wait);
+              if (!ok) *abort_flag = 1;
               asm volatile("fence.proxy.async.global;" ::: "memory");
             }
-            mbar_arrive_tx(&full[s], XB + TC_B_BYTES);
+            // (issued even after a failed wait, so that the stage's barrier
+            // completes and is drained below; nobody reads it then)
             tma_load_2d(smem_u32(xd), &tm_gt, &full[s], e * TC_BK, ti.mb * BMT);
-            tma_load_2d(smem_u32(bd), &tm_bpt, &full[s], e * TC_BK, ti.nb * TC_BN);
           }
           ++issued;
           if (++s == NST) {
@@ -388,7 +409,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       int last_s = -1;      // stage (and its phase) of the last commit
       uint32_t last_ph = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int tile = t_first; tile < ntiles && ok; tile += t_step) {
         const TileInfo ti = tile_info(a, tile);
         ok = mbar_wait(&acc_empty[buf], aph[buf] ^ 1, abort_flag, a.hdr);
         if (!ok) break;
@@ -449,7 +470,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     int buf = 0;
     uint32_t aph[2] = {0, 0};
     bool ok = true;
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+    for (int tile = t_first; tile < ntiles && ok; tile += t_step) {
       const TileInfo ti = tile_info(a, tile);
       ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], aph[buf], abort_flag, a.hdr));
       if (!ok) break;
@@ -468,7 +489,121 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int row = q * 32 + lane;
       const int m = ti.mb * BMT + h * TC_BM + row;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NH + h) * 256;
-      if (ti.kind == 0) {
+      // K parts (S > 1): every part puts its accumulator in the workspace and
+      // raises its flag; then each part sums, in part order, its share of the
+      // tile (a projection tile whole on part 0, 256 / S output channels per
+      // part) back into its own accumulator, and the code below stores that
+      // share.  A warp's partial is [column / 4][lane][4] fp32 (a store of 4
+      // columns is 512 contiguous bytes, a run of columns one contiguous
+      // block), read back with one bulk copy per part and chunk of columns
+      // into the ring, which is idle once the accumulator is complete (a CTA
+      // holds one tile when S > 1).  A warp whose 32 rows are all past M skips
+      // the exchange on every part alike.
+      int lo = 0, hi = TC_BN;
+      bool run_gate = true;
+      if (BMT == 128 && a.S > 1) {
+        const int part = (int)(blockIdx.x % (unsigned)a.S);
+        const bool rows = ti.mb * BMT + h * TC_BM + q * 32 < a.M;
+        const int ncol = ti.kind == 0 ? a.NE : TC_BN;
+        constexpr int QF = TC_BN * 32;  // floats of one warp's partial
+        const float* qbase = a.kpart + ((size_t)tile * a.S * 4 * NH + 4 * h + q) * QF;
+        int* kflag = a.kflags + (tile * a.S) * 4 * NH + 4 * h + q;
+        if (rows) {
+          float4* pdst = reinterpret_cast<float4*>(const_cast<float*>(qbase) + (size_t)part * 4 * NH * QF);
+          for (int c0 = 0; c0 < ncol; c0 += 16) {
+            float v[16];
+            tmem_ld16(taddr + c0, v);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              pdst[(c0 / 4 + i) * 32 + lane] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          }
+          // the warp barrier orders every lane's stores before lane 0's release
+          __syncwarp();
+          if (lane == 0) st_release_gpu(kflag + part * 4 * NH, epoch + 1);
+        }
+        lo = ti.kind == 0 ? 0 : part * (TC_BN / a.S);
+        hi = !rows ? lo : ti.kind == 0 ? (part == 0 ? a.NE : 0) : lo + TC_BN / a.S;
+        run_gate = part == 0;
+        if (hi > lo) {
+          // this warp's share of the ring (split among the warps that hold
+          // rows, warps 0 .. nw - 1): NB buffers of S x CC columns, then NB
+          // mbarriers.  CC columns per chunk: the whole share when it fits.
+          const int nw = min(4, (a.M - ti.mb * BMT - h * TC_BM + 31) / 32);
+          const int XW = (NST * tc_stage_bytes(BMT) / nw) & ~1023;
+          uint8_t* xw = smem + q * XW;
+          uint64_t* xbar = reinterpret_cast<uint64_t*>(xw + XW - 128);
+          int CC = hi - lo;
+          while (a.S * CC * 128 > XW - 128) CC = (CC / 2 + 15) & ~15;
+          const int CB = a.S * CC * 128;  // bytes of one buffer
+          const int nch = (hi - lo + CC - 1) / CC;
+          const int NB = min(min(nch, (XW - 128) / CB), 16);
+          if (lane == 0) {
+            for (int b = 0; b < NB; ++b) mbar_init(&xbar[b], 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+          }
+          // lane p watches part p's flag: one round trip per poll for all parts
+          const bool fok = lane >= a.S || wait_flag_eq(kflag + lane * 4 * NH, epoch + 1, a.hdr);
+          if (!__all_sync(0xffffffffu, fok)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          auto issue = [&](int ch) {  // lane 0: columns lo + CC ch .. of every part
+            const int b = ch % NB, c0 = lo + ch * CC, nb = (min(hi, c0 + CC) - c0) * 128;
+            mbar_arrive_tx(&xbar[b], a.S * nb);
+            for (int p = 0; p < a.S; ++p)
+              bulk_g2s(xw + b * CB + p * CC * 128, qbase + (size_t)p * 4 * NH * QF + c0 * 32, nb, &xbar[b]);
+          };
+          // the polling lanes' acquires, the warp barrier, then lane 0's bulk
+          // copies (async proxy) read the partials
+          __syncwarp();
+          if (lane == 0) {
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            for (int ch = 0; ch < NB; ++ch) issue(ch);
+          }
+          int ch = 0;
+          for (; ch < nch; ++ch) {
+            const int b = ch % NB, c0 = lo + ch * CC, c1 = min(hi, c0 + CC);
+            if (!__all_sync(0xffffffffu, mbar_wait(&xbar[b], (ch / NB) & 1, abort_flag, a.hdr))) break;
+            for (int g = c0; g < c1; g += 16) {
+              float sum[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) sum[i] = 0.f;
+#pragma unroll
+              for (int p = 0; p < 8; ++p) {
+                if (p >= a.S) break;
+                const float4* src = reinterpret_cast<const float4*>(xw + b * CB + p * CC * 128 + (g - c0) * 128) + lane;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float4 v = src[32 * i];
+                  sum[4 * i] += v.x;
+                  sum[4 * i + 1] += v.y;
+                  sum[4 * i + 2] += v.z;
+                  sum[4 * i + 3] += v.w;
+                }
+              }
+              tmem_st16(taddr + g, sum);
+            }
+            __syncwarp();
+            if (lane == 0 && ch + NB < nch) {
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+              issue(ch + NB);
+            }
+          }
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+          if (ch < nch) {
+            // gave up: let the copies in flight land before the ring is released
+            if (lane == 0)
+              for (int c = ch; c < nch && c < ch + NB; ++c) tc_drain(&xbar[c % NB], (c / NB) & 1);
+            __syncwarp();
+            ok = false;
+            break;
+          }
+        }
+      }
+      if (ti.kind == 0 && !run_gate) {
+        // another part runs this projection tile's gate
+      } else if (ti.kind == 0) {
         // projection tile: columns 0..r-1 = t, column r = gate logit
         __nv_bfloat16* gdst = a.gt + (size_t)m * a.r;
         float g;
@@ -549,15 +684,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const unsigned below = __ballot_sync(0xffffffffu, valid && g < a.tau);
         if (lane == 0 && a.mask_count && below) atomicAdd(&a.hdr->ec_done, __popc(below));
         asm volatile("fence.proxy.async.global;" ::: "memory");
-        __threadfence();
         tc_fence_before();
+        // the warp barrier orders every lane's gt stores before lane 0's release
         __syncwarp();
         // one flag per epilogue warp (32 token rows), tagged with this launch's epoch
         if (lane == 0) st_release_gpu(&a.mflags[4 * NH * ti.mb + 4 * h + q], epoch + 1);
       } else {
         const int n0 = ti.nb * TC_BN;
 #pragma unroll 1
-        for (int c0 = 0; c0 < TC_BN; c0 += 32) {
+        for (int c0 = lo; c0 < hi; c0 += 32) {
           float v[32];
           tmem_ld32(taddr + c0, v);
           if (!GROUP) {
@@ -591,14 +726,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+    for (int tile = t_first; tile < ntiles && ok; tile += t_step) {
       const TileInfo ti = tile_info(a, tile);
-      const int KT = a.K / TC_BK;
       for (int k = 0; k < ti.steps && ok; ++k) {
         ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, a.hdr));
         if (!ok) break;
-        if (ti.kind == 1 && k < KT) {
-          dequant_tile<GROUP>(ps + s * TC_P_BYTES, bs + s * TC_B_BYTES, dt, a, ti.nb, k);
+        if (ti.kind == 1 && k < ti.nk) {
+          dequant_tile<GROUP>(ps + s * TC_P_BYTES, bs + s * TC_B_BYTES, dt, a, ti.nb, ti.k0 + k);
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
         __syncwarp();
@@ -654,7 +788,8 @@ static int launch_tc_t(const TcPlan& p, const TcArgs& a, const CUtensorMap* maps
   });
   if (attr_err != cudaSuccess) return set_cuda_error("cudaFuncSetAttribute(tc)", attr_err);
   const int ntiles = (a.with_ec ? a.Mb : 0) + a.Mb * a.Nb;
-  const int grid = ntiles < p.grid ? ntiles : p.grid;
+  const int groups = ntiles < p.grid / a.S ? ntiles : p.grid / a.S;
+  const int grid = groups * a.S;
   const size_t smem = tc_smem(a.nst, BMT) + (a.gate_kind == 1 ? tc_gpar_bytes(a.gate_h, a.r) : 0);
   tc_kernel<GROUP, BMT><<<grid, TC_THREADS, smem, st>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4]);
   cudaError_t e = cudaGetLastError();
@@ -671,7 +806,8 @@ static int tc_tile_rows(int M, const LayerView& L, bool with_ec) {
 }
 
 int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M, __nv_bfloat16* y, bool with_ec,
-              WsHeader* hdr, int* mflags, __nv_bfloat16* gt, float* gate_out, int* mask_count, cudaStream_t st) {
+              WsHeader* hdr, int* mflags, int* kflags, float* kpart, __nv_bfloat16* gt, float* gate_out,
+              int* mask_count, cudaStream_t st) {
   if (L.N % TC_BN) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "tensor-core path needs N %% 256 == 0 (N=%d)", L.N);
   const int bmt = tc_tile_rows(M, L, with_ec);
   TcArgs a = {};
@@ -702,6 +838,17 @@ int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
   a.gb2 = L.gb2;
   a.alpha = L.alpha;
   a.nst = bmt == 256 ? 3 : (a.gate_kind == 1 ? TC_STAGES - 1 : TC_STAGES);
+  // K parts at mid M: while the tiles fill less than half the SMs, split each
+  // tile's K in two more parts (up to 8, at least 8 k-steps per part); every
+  // group of S CTAs then holds exactly one tile, all resident at once
+  a.S = 1;
+  a.kflags = kflags;
+  a.kpart = kpart;
+  if (bmt == 128 && kflags && kpart) {
+    const int ntiles = (a.with_ec ? a.Mb : 0) + a.Mb * a.Nb;
+    const int KT = L.K / TC_BK;
+    while (a.S < 8 && ntiles * a.S * 2 <= p.grid && KT % (a.S * 2) == 0 && KT / (a.S * 2) >= 8) a.S *= 2;
+  }
   const TestFault tf_ = test_fault();
   a.tag_skew = tf_.kernel == 2 ? 1 : 0;
   a.pub_wait = tf_.kernel == 2 ? tf_.cycles : kWaitCycles;
