@@ -333,8 +333,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tma_load_2d(smem_u32(bd), &tm_agt, &full[s], (ti.k0 + k) * TC_BK, 0);
           } else if (k < ti.nk) {
             const int kg = ti.k0 + k;
-            // warm L2 a few k-steps ahead so the shallow shared-memory ring
-            // does not see the full HBM latency on every stage
+            mbar_arrive_tx(&full[s], XB + TC_P_BYTES);
+            tma_load_2d(smem_u32(xd), &tm_x, &full[s], kg * TC_BK, ti.mb * BMT);
+            tma_load_3d(smem_u32(pd), &tm_w, &full[s], 0, kg, ti.nb * (TC_BN / 16));
+            // then warm L2 a few k-steps ahead (each TMA instruction costs this
+            // thread tens of ns, so the step's own loads go out first), so the
+            // shallow shared-memory ring does not see the full HBM latency on
+            // every stage
             if (k + TC_PREFETCH < ti.nk) {
               tma_prefetch_2d(&tm_x, (kg + TC_PREFETCH) * TC_BK, ti.mb * BMT);
               tma_prefetch_3d(&tm_w, 0, kg + TC_PREFETCH, ti.nb * (TC_BN / 16));
@@ -357,14 +362,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 }
               }
             }
-            if (k == 0)
-              for (int pk = 1; pk < TC_PREFETCH && pk < ti.nk; ++pk) {
+            // the CTA's first tile: once the ring's first loads are out, warm the
+            // steps after them that the per-step warm-up above does not reach
+            // (later tiles had theirs warmed during the previous tile's tail)
+            if (tile == t_first && k == min(NST, ti.nk) - 1)
+              for (int pk = NST; pk < TC_PREFETCH && pk < ti.nk; ++pk) {
                 tma_prefetch_2d(&tm_x, (ti.k0 + pk) * TC_BK, ti.mb * BMT);
                 tma_prefetch_3d(&tm_w, 0, ti.k0 + pk, ti.nb * (TC_BN / 16));
               }
-            mbar_arrive_tx(&full[s], XB + TC_P_BYTES);
-            tma_load_2d(smem_u32(xd), &tm_x, &full[s], kg * TC_BK, ti.mb * BMT);
-            tma_load_3d(smem_u32(pd), &tm_w, &full[s], 0, kg, ti.nb * (TC_BN / 16));
           } else {
             const int e = k - ti.nk;
             // B' does not depend on the projection: its load goes out first
@@ -569,9 +574,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               float sum[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i) sum[i] = 0.f;
-#pragma unroll
-              for (int p = 0; p < 8; ++p) {
-                if (p >= a.S) break;
+              for (int p = 0; p < a.S; ++p) {
                 const float4* src = reinterpret_cast<const float4*>(xw + b * CB + p * CC * 128 + (g - c0) * 128) + lane;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
