@@ -78,10 +78,12 @@ struct D3Args {
 
 // Shared-memory carve-up (same on host and device).
 struct D3Smem {
-  uint32_t units, bps, scs, ts, gts, gpart, gv, rg, stage, bars, total;
+  uint32_t units, bps, scs, ts, gts, gpart, gv, rg, gp, stage, bars, total;
 };
 __host__ __device__ __forceinline__ uint32_t d3_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
-__host__ __device__ __forceinline__ D3Smem d3_smem(int MT, int ubytes, int own_cap, int r, int gate_kind) {
+// rank-gate parameters W1 [h][r], W2 [r][h], b1 [h], b2 [r] fp32, staged at kernel start
+__host__ __device__ __forceinline__ uint32_t d3_gp_bytes(int r, int h) { return (uint32_t)(2 * h * r + h + r) * 4; }
+__host__ __device__ __forceinline__ D3Smem d3_smem(int MT, int ubytes, int own_cap, int r, int gate_kind, int gate_h) {
   D3Smem s;
   uint32_t off = 0;
   s.units = off;  // the CTA's units, each at a 1024-byte boundary
@@ -100,6 +102,8 @@ __host__ __device__ __forceinline__ D3Smem d3_smem(int MT, int ubytes, int own_c
   off += 64;
   s.rg = off;  // rank gate: hidden [MT][32] and gamma [MT][r] fp32
   off += gate_kind == 1 ? d3_up(MT * (32 + r) * 4, 16) : 0;
+  s.gp = off;  // rank gate: its parameters (16-byte multiples: h in {8, 16, 32}, r a multiple of 16)
+  off += gate_kind == 1 ? d3_gp_bytes(r, gate_h) : 0;
   s.stage = off;  // per warp [MT tokens][16 channels] bf16
   off += D3_NW * MT * 32;
   s.bars = off;  // unit barriers, partials complete, epilogue operands, fetched t, gt ready
@@ -347,11 +351,44 @@ __device__ __forceinline__ uint32_t atom_add_acqrel_cta(int* p, int v) {
 // logits are in shared memory), then the reported gate and mask count (CTA 0).
 // Scalar gate: g = sigmoid(logit + b_g), gt = bf16(g t).  The pages' per-rank
 // gate: u = relu(W1 t + b1), gamma = sigmoid(W2 u + b2), gt = bf16(alpha gamma t),
-// reported gate = mean of gamma (summed in rank order).  Padded tokens get
-// zero rows.
+// reported gate = mean of gamma (a fixed lane-strided then shuffle-tree
+// order).  Padded tokens get zero rows.
+//
+// What the gate builder reads of the launch's arguments, passed by value: an
+// out-of-line callee reading the kernel's parameter block through a reference
+// paid microseconds of load latency before its first instruction of work.
+struct D3Gate {
+  float* gate_out;
+  int* mask_count;
+  WsHeader* hdr;
+  const float *gw1, *gb1, *gw2, *gb2;
+  int M, r, gate_kind, gate_h, ubytes, own_cap;
+  float b_g, alpha, tau;
+};
+__device__ __forceinline__ D3Gate d3_gate_args(const D3Args& a) {
+  D3Gate g;
+  g.gate_out = a.gate_out;
+  g.mask_count = a.mask_count;
+  g.hdr = a.hdr;
+  g.gw1 = a.gw1;
+  g.gb1 = a.gb1;
+  g.gw2 = a.gw2;
+  g.gb2 = a.gb2;
+  g.M = a.M;
+  g.r = a.r;
+  g.gate_kind = a.gate_kind;
+  g.gate_h = a.gate_h;
+  g.ubytes = a.ubytes;
+  g.own_cap = a.own_cap;
+  g.b_g = a.b_g;
+  g.alpha = a.alpha;
+  g.tau = a.tau;
+  return g;
+}
+
 template <int MT>
-__device__ __noinline__ void d3_build_gate(const D3Args& a, uint8_t* sm) {
-  const D3Smem SL = d3_smem(MT, a.ubytes, a.own_cap, a.r, a.gate_kind);
+__device__ __noinline__ void d3_build_gate(const D3Gate a, uint8_t* sm, volatile int* abortp) {
+  const D3Smem SL = d3_smem(MT, a.ubytes, a.own_cap, a.r, a.gate_kind, a.gate_h);
   const float* ts = reinterpret_cast<const float*>(sm + SL.ts);
   __nv_bfloat16* gts = reinterpret_cast<__nv_bfloat16*>(sm + SL.gts);
   float* gv = reinterpret_cast<float*>(sm + SL.gv);
@@ -370,45 +407,87 @@ __device__ __noinline__ void d3_build_gate(const D3Args& a, uint8_t* sm) {
     const int h = a.gate_h, r = a.r;
     float* hid = reinterpret_cast<float*>(sm + SL.rg);  // [MT][32]
     float* gam = hid + MT * 32;                         // [MT][r]
-    for (int idx = tid; idx < a.M * h; idx += D3_THREADS) {
-      const int m = idx / h, i = idx - m * h;
-      const float4* w1 = reinterpret_cast<const float4*>(a.gw1 + (size_t)i * r);
-      const float4* tv = reinterpret_cast<const float4*>(ts + m * r);
-      float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
-      for (int j4 = 0; j4 < r / 4; ++j4) {
-        const float4 wv = __ldg(w1 + j4), xv = tv[j4];
-        z0 = fmaf(wv.x, xv.x, z0);
-        z1 = fmaf(wv.y, xv.y, z1);
-        z2 = fmaf(wv.z, xv.z, z2);
-        z3 = fmaf(wv.w, xv.w, z3);
+    // the parameters, staged in shared memory at kernel start (long landed:
+    // the wait returns at once; a failed wait only leaves this CTA's gate
+    // unused, the strips' own waits then stop)
+    const float* gp = reinterpret_cast<const float*>(sm + SL.gp);
+    const float* W1 = gp;
+    const float* W2 = gp + h * r;
+    const float* B1 = gp + 2 * h * r;
+    const float* B2 = B1 + h;
+    d3_wait(reinterpret_cast<uint64_t*>(sm + SL.bars) + 2 * D3_MAXU, 0, abortp, a.hdr);
+    // u = relu(W1 t + b1): a team of tpi threads (a power of two, as many as
+    // the block holds) per (token, hidden) item, each over j = sub, sub + tpi,
+    // ... started at an item-dependent offset so that a warp's W1 and t reads
+    // fall in different banks, then a fixed shuffle tree over the team
+    {
+      const int items = a.M * h;
+      int tpi = 32;
+      while (tpi > 1 && (tpi * items > D3_THREADS || r % tpi)) tpi >>= 1;
+      for (int base = 0; base < items * tpi; base += D3_THREADS) {
+        const int idx = base + tid, item = idx / tpi, sub = idx - item * tpi;
+        float z = 0.f;
+        if (item < items) {
+          const int m = item / h, i = item - m * h;
+          const float* w1 = W1 + i * r;
+          const float* tv = ts + m * r;
+          // j = sub + tpi (i + k) mod r for k = 0, 1, ...: every j = sub mod tpi
+          // once (tpi divides r), from an item-dependent start, wrapped by a
+          // subtraction rather than a division; two alternating sums
+          const int n = r / tpi;
+          int j = (i * tpi) % r + sub;
+          float z0 = 0.f, z1 = 0.f;
+          for (int k = 0; k < n; k += 2) {
+            z0 = fmaf(w1[j], tv[j], z0);
+            j += tpi;
+            if (j >= r) j -= r;
+            if (k + 1 < n) {
+              z1 = fmaf(w1[j], tv[j], z1);
+              j += tpi;
+              if (j >= r) j -= r;
+            }
+          }
+          z = z0 + z1;
+        }
+        for (int o = tpi >> 1; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        if (item < items && sub == 0) {
+          const int m = item / h, i = item - m * h;
+          hid[m * 32 + i] = fmaxf(z + B1[i], 0.f);
+        }
       }
-      hid[m * 32 + i] = fmaxf((z0 + z1) + (z2 + z3) + __ldg(a.gb1 + i), 0.f);
     }
     __syncthreads();
+    // gamma = sigmoid(W2 u + b2), gt = bf16(alpha gamma t): one thread per
+    // (token, rank) item, its W2 row and u read from an item-dependent offset
     for (int idx = tid; idx < MT * r; idx += D3_THREADS) {
       const int m = idx / r, j = idx - m * r;
       float gam_v = 0.f;
       if (m < a.M) {
-        const float4* w2 = reinterpret_cast<const float4*>(a.gw2 + (size_t)j * h);
-        const float4* uv = reinterpret_cast<const float4*>(hid + m * 32);
-        float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
-        for (int i4 = 0; i4 < h / 4; ++i4) {
-          const float4 wv = __ldg(w2 + i4), xv = uv[i4];
-          z0 = fmaf(wv.x, xv.x, z0);
-          z1 = fmaf(wv.y, xv.y, z1);
-          z2 = fmaf(wv.z, xv.z, z2);
-          z3 = fmaf(wv.w, xv.w, z3);
+        const float* w2 = W2 + j * h;
+        const float* uv = hid + m * 32;
+        float z0 = 0.f, z1 = 0.f;
+        for (int k = 0; k < h; k += 2) {
+          const int i0 = (k + j) & (h - 1), i1 = (k + 1 + j) & (h - 1);
+          z0 = fmaf(w2[i0], uv[i0], z0);
+          z1 = fmaf(w2[i1], uv[i1], z1);
         }
-        gam_v = sigmoidf_(__ldg(a.gb2 + j) + ((z0 + z1) + (z2 + z3)));
+        gam_v = sigmoidf_(B2[j] + (z0 + z1));
       }
       gam[m * r + j] = gam_v;
       gts[m * gs + j] = __float2bfloat16_rn(m < a.M ? a.alpha * gam_v * ts[m * r + j] : 0.f);
     }
     __syncthreads();
-    if (tid < MT) {
-      float sgm = 0.f;
-      for (int j = 0; j < r; ++j) sgm += gam[tid * r + j];
-      gv[tid] = tid < a.M ? sgm / (float)r : 0.f;
+    // g = mean of gamma: warp m sums token m's r values (lane-strided, then a
+    // fixed shuffle tree)
+    {
+      const int warp = tid >> 5, lane = tid & 31;
+      if (warp < MT) {
+        float sgm = 0.f;
+        for (int j = lane; j < r; j += 32) sgm += gam[warp * r + j];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sgm += __shfl_xor_sync(0xffffffffu, sgm, o);
+        if (lane == 0) gv[warp] = warp < a.M ? sgm / (float)r : 0.f;
+      }
     }
   }
   __syncthreads();
@@ -430,7 +509,7 @@ template <int MT, bool GROUP>
 __device__ __noinline__ void d3_finish_strip(const D3Args& a, uint8_t* sm, int j, int p, const uint8_t* ubase, int CH,
                                              int lane, int warp) {
   constexpr int NT = MT / 8;
-  const D3Smem SL = d3_smem(MT, a.ubytes, a.own_cap, a.r, a.gate_kind);
+  const D3Smem SL = d3_smem(MT, a.ubytes, a.own_cap, a.r, a.gate_kind, a.gate_h);
   const __nv_bfloat16* bps = reinterpret_cast<const __nv_bfloat16*>(sm + SL.bps);
   const __half* scs = reinterpret_cast<const __half*>(sm + SL.scs);
   const __nv_bfloat16* gts = reinterpret_cast<const __nv_bfloat16*>(sm + SL.gts);
@@ -527,7 +606,7 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ int s_abort, s_eccnt, s_fetched;
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const D3Smem SL = d3_smem(MT, a.ubytes, a.own_cap, a.r, a.gate_kind);
+  const D3Smem SL = d3_smem(MT, a.ubytes, a.own_cap, a.r, a.gate_kind, a.gate_h);
   uint8_t* units = sm + SL.units;
   __nv_bfloat16* bps = reinterpret_cast<__nv_bfloat16*>(sm + SL.bps);
   __half* scs = reinterpret_cast<__half*>(sm + SL.scs);
@@ -568,7 +647,9 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncwarp();
     // epilogue operands of the CTA's strips: B' rows and per-channel scales
-    const uint32_t epi_bytes = (uint32_t)n_w * ((has_ec ? 32u * a.r : 0u) + (GROUP ? 0u : 32u));
+    // (and the rank gate's parameters, which every CTA's gate builder reads)
+    const uint32_t gp_bytes = has_ec && a.gate_kind == 1 ? d3_gp_bytes(a.r, a.gate_h) : 0u;
+    const uint32_t epi_bytes = (uint32_t)n_w * ((has_ec ? 32u * a.r : 0u) + (GROUP ? 0u : 32u)) + gp_bytes;
     if (lane == 0) {
       if (epi_bytes)
         mbar_arrive_tx(epibar, epi_bytes);
@@ -576,6 +657,14 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
         mbar_arrive(epibar);
     }
     __syncwarp();
+    if (gp_bytes && lane < 4) {
+      const int h = a.gate_h, r = a.r;
+      float* gp = reinterpret_cast<float*>(sm + SL.gp);
+      const float* src = lane == 0 ? a.gw1 : lane == 1 ? a.gw2 : lane == 2 ? a.gb1 : a.gb2;
+      const int off = lane == 0 ? 0 : lane == 1 ? h * r : lane == 2 ? 2 * h * r : 2 * h * r + h;
+      const int n = lane < 2 ? h * r : lane == 2 ? h : r;
+      bulk_g2s(gp + off, src, (uint32_t)n * 4, epibar);
+    }
     for (int j = lane; j < n_w; j += 32) {
       const int p = w_lo + j;
       if (has_ec) tma_load_2d(smem_u32(bps + (size_t)j * 16 * a.r), &tm_bp, epibar, 0, 16 * p);
@@ -842,7 +931,7 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
     // Read once by every thread between two barriers: nothing writes the flag
     // before the gate block's last barrier, so the branch below is uniform.
     live = !*abortp;
-    if (needs_t && live) d3_build_gate<MT>(a, sm);
+    if (needs_t && live) d3_build_gate<MT>(d3_gate_args(a), sm, abortp);
   }
   if (live) {
     // strip j by warp j % 16, as soon as its 16 partials (and gt) are ready
@@ -881,7 +970,7 @@ struct D3Plan {
   std::vector<short4> tab;
 };
 
-static D3Plan make_d3_plan(int MT, int K, int N, int r, int group, int gate_kind, int sms) {
+static D3Plan make_d3_plan(int MT, int K, int N, int r, int group, int gate_kind, int gate_h, int sms) {
   D3Plan p = {};
   p.MT = MT;
   p.why = nullptr;
@@ -934,7 +1023,7 @@ static D3Plan make_d3_plan(int MT, int K, int N, int r, int group, int gate_kind
   }
   p.own_cap = own;
   p.ubytes = ub;
-  p.smem = d3_smem(MT, ub, own, r, gate_kind).total;
+  p.smem = d3_smem(MT, ub, own, r, gate_kind, gate_h).total;
   if (p.smem > D3_SMEM_MAX) p.why = "a CTA's share does not fit in shared memory";
   return p;
 }
@@ -953,22 +1042,22 @@ static cudaError_t d3_attrs(size_t smem) {
 }
 
 // The plan for a shape (cached per device).
-static const D3Plan& d3_plan(int MT, int K, int N, int r, int group, int gate_kind, int sms) {
+static const D3Plan& d3_plan(int MT, int K, int N, int r, int group, int gate_kind, int gate_h, int sms) {
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int, int, int, int, int, int>, D3Plan> cache;
+  static std::map<std::tuple<int, int, int, int, int, int, int, int, int>, D3Plan> cache;
   int dev = 0;
   cudaGetDevice(&dev);
-  const auto key = std::make_tuple(dev, MT, K, N, r, group, gate_kind, sms);
+  if (gate_kind != 1) gate_h = 0;
+  const auto key = std::make_tuple(dev, MT, K, N, r, group, gate_kind, gate_h, sms);
   std::lock_guard<std::mutex> lk(mu);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
-  return cache.emplace(key, make_d3_plan(MT, K, N, r, group, gate_kind, sms)).first->second;
+  return cache.emplace(key, make_d3_plan(MT, K, N, r, group, gate_kind, gate_h, sms)).first->second;
 }
 
 const char* decode3_unsupported(int M, int K, int N, int r, int group, int gate_kind, int gate_h) {
-  (void)gate_h;
   if (M < 1 || M > 16) return "the decode kernel needs 1 <= M <= 16";
-  return d3_plan(M <= 8 ? 8 : 16, K, N, r, group, r > 0 ? gate_kind : 0, device_sm_count()).why;
+  return d3_plan(M <= 8 ? 8 : 16, K, N, r, group, r > 0 ? gate_kind : 0, gate_h, device_sm_count()).why;
 }
 
 template <int MT, int CH, bool GROUP>
@@ -1018,7 +1107,7 @@ int launch_decode3(const LayerView& Lv, const __nv_bfloat16* x, int M, __nv_bflo
   if (M < 1 || M > 16) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path needs 1 <= M <= 16 (M=%d)", M);
   const int MT = M <= 8 ? 8 : 16;
   const int gk = Lv.r > 0 ? Lv.gate_kind : 0;
-  const D3Plan& p = d3_plan(MT, Lv.K, Lv.N, Lv.r, Lv.group, gk, device_sm_count());
+  const D3Plan& p = d3_plan(MT, Lv.K, Lv.N, Lv.r, Lv.group, gk, Lv.gate_h, device_sm_count());
   if (p.why) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: %s", p.why);
   if (ec_only && Lv.r == 0) return set_error(SPEAR_ERR_INVALID_ARG, "EC-only launch without an EC");
   if (MT == 8 && p.CH < 1) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "decode path: K too small");
