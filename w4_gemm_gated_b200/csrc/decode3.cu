@@ -568,11 +568,21 @@ __device__ __noinline__ void d3_finish_strip(const D3Args& a, uint8_t* sm, int j
 
 // Whether every EC item of this launch is published (each lane checks every
 // flag itself, with acquire ordering for its own later reads of the rows).
+// Every EC item's flag at this launch's tag?  Lane e reads flag e (all in
+// flight together, one round trip), the warp votes, and once all are set each
+// lane's acquire fence orders the rows read after it.
 __device__ __forceinline__ bool d3_flags_ready(const D3Args& a, int tag) {
-  const int ne = a.ES + a.gate_item;
-  bool ready = true;
-  for (int e = 0; e < ne; ++e) ready = ready && ld_acquire_gpu(&a.hdr->d3_flag[e]) == tag + a.tag_skew;
-  return __all_sync(0xffffffffu, ready);
+  const int ne = a.ES + a.gate_item;  // <= D3_MAXE <= 32
+  bool mine = true;
+  if ((int)(threadIdx.x & 31) < ne) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(&a.hdr->d3_flag[threadIdx.x & 31]) : "memory");
+    mine = v == tag + a.tag_skew;
+  }
+  const bool all = __all_sync(0xffffffffu, mine);
+  if (all) asm volatile("fence.acq_rel.gpu;" ::: "memory");
+  __syncwarp();
+  return all;
 }
 
 // The published rows of the live tokens into shared memory by cp.async, one
@@ -842,7 +852,7 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
         for (int w2 = 0; w2 < D3_NW; ++w2) g += gpart[w2 * MT + lane];
         dst[lane * 16] = g;
       }
-      __threadfence();
+      // the warp barrier orders every lane's rows before lane 0's release
       __syncwarp();
       if (lane == 0) st_release_gpu(&a.hdr->d3_flag[ec_item], tag);
     }
