@@ -59,6 +59,7 @@ struct D3Args {
   WsHeader* hdr;
   float* tf;                // [D3_MAXE][MT][16] fp32: published EC rows (t, then the gate logit in row 0)
   const float *gw1, *gb1, *gw2, *gb2;
+  const uint8_t* gate_row;   // row r of [A^T ; w_g]: w_g over all of K, bf16 (the gate item's one unit)
   int M, K, N, r;
   float b_g, tau, alpha;
   int G;                    // CTAs
@@ -681,6 +682,21 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
       if (!GROUP) bulk_g2s(scs + j * 16, a.scales + 16 * p, 32, epibar);
     }
     // every unit: nothing here depends on the previous kernel in the stream.
+    // The EC item's units go first: the rows it publishes are on every CTA's
+    // critical path.  An A^T unit (k-tile u of every warp's slice of a
+    // 16-row strip) is one 32 KB box of a 3-D map [slice][row][k]; the gate
+    // row is one contiguous run (TMA instructions cost the issuing thread tens
+    // of ns each, so 16 small boxes per unit delayed the EC item).
+    for (int u = lane; u < n_ecu; u += 32) {
+      uint64_t* bar = &ubar[u];
+      if (ec_item < a.ES) {
+        mbar_arrive_tx(bar, D3_ECU);
+        tma_load_3d(smem_u32(ubase(u)), &tm_agt, bar, u * 64, 16 * ec_item, 0);
+      } else {
+        mbar_arrive_tx(bar, D3_NW * CH * 128);
+        bulk_g2s(ubase(u), a.gate_row, D3_NW * CH * 128, bar);
+      }
+    }
     // A weight unit (strip p, all of K) is one contiguous run of the packed
     // array: it goes as 1-D bulk copies of 8 KB issued from several lanes
     // (measured much faster per SM than one large tensor box).
@@ -692,22 +708,6 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
       const int p = w_lo + (u - n_ecu);
       bulk_g2s(ubase(u) + k * PIECE, a.w + ((size_t)p * KT * 512 + (size_t)k * PIECE), PIECE, &ubar[u]);
       if (GROUP && k == 0) tma_load_2d(smem_u32(ubase(u)) + KT * 512, &tm_gs, &ubar[u], 16 * p, 0);
-    }
-    for (int u = lane; u < n_ecu; u += 32) {
-      uint64_t* bar = &ubar[u];
-      const uint32_t dst = smem_u32(ubase(u));
-      {
-        if (ec_item < a.ES) {
-          // k-tile u of every warp's slice of A^T strip ec_item
-          mbar_arrive_tx(bar, D3_ECU);
-          for (int wi = 0; wi < D3_NW; ++wi)
-            tma_load_2d(dst + wi * 2048, &tm_agt, bar, (wi * CH + u) * 64, 16 * ec_item);
-        } else {
-          // the gate row over every warp's slice
-          mbar_arrive_tx(bar, D3_NW * CH * 128);
-          for (int wi = 0; wi < D3_NW; ++wi) tma_load_2d(dst + wi * CH * 128, &tm_gate, bar, wi * CH * 64, a.r);
-        }
-      }
     }
   }
   if (warp == 1) {
@@ -1110,6 +1110,22 @@ static int d3_dispatch_c(int ch, bool group, const D3Args& a, const CUtensorMap*
   }
 }
 
+// [A^T ; w_g] ((r + 1) rows of K bf16) as a 3-D array [warp slice][row][k in
+// the slice]: box (64 k, 16 rows, 16 slices) = k-tile u of every warp's slice
+// of one 16-row strip, landing as [slice][row][64 k] with the 128-byte swizzle
+// of the per-slice 2 KB tiles the EC item reads.
+static bool d3_tmap_agt(CUtensorMap* m, const void* agt, int K, int r, int CH) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)CH * 64, (cuuint64_t)r + 1, (cuuint64_t)D3_NW};
+  const cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)CH * 128};
+  const cuuint32_t box[3] = {64, 16, D3_NW};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(agt), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 size_t decode3_tf_bytes() { return (size_t)D3_MAXE * 16 * 16 * sizeof(float); }
 
 int launch_decode3(const LayerView& Lv, const __nv_bfloat16* x, int M, __nv_bfloat16* y, WsHeader* hdr, void* tf,
@@ -1163,9 +1179,9 @@ int launch_decode3(const LayerView& Lv, const __nv_bfloat16* x, int M, __nv_bflo
   const int KT = Lv.K / 64;
   bool ok = tmap_packed_box(&maps[0], Lv.w, Lv.K, Lv.N, KT, 1);
   if (ok && a.ES > 0) {
-    ok = tmap_2d_bf16(&maps[1], Lv.agt, Lv.K, Lv.r + 1, 64, 16);
-    if (ok) ok = tmap_2d_bf16(&maps[2], Lv.agt, Lv.K, Lv.r + 1, 64 * p.CH, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok = d3_tmap_agt(&maps[1], Lv.agt, Lv.K, Lv.r, p.CH);
     if (ok) ok = tmap_2d_bf16(&maps[3], Lv.bpt, Lv.r, Lv.N, Lv.r, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+    a.gate_row = reinterpret_cast<const uint8_t*>(Lv.agt) + (size_t)Lv.r * Lv.K * 2;
   }
   if (ok && Lv.group) ok = tmap_2d_f16(&maps[4], Lv.scales, Lv.N, Lv.K / 128, 16, KT / 2);
   if (!ok) return set_error(SPEAR_ERR_CUDA, "cuTensorMapEncodeTiled failed (decode)");
