@@ -1,8 +1,9 @@
 """GPU parity of the tensor-core kernel's K parts at mid M, against the CPU
 oracle.
 
-While the tiles of a launch fill less than half the SMs, the kernel splits
-every tile's K into S = 2, 4 or 8 parts (at least 8 k-steps each), one CTA per
+While the 128-token tiles of a launch fill less than half the SMs (256-token
+tiles are taken only where they fill at least half), the kernel splits every
+tile's K into S = 2, 4 or 8 parts (at least 8 k-steps each), one CTA per
 part.  Every part puts its fp32 accumulator in the workspace; each then sums,
 in part order, its 256 / S output channels (the projection tile whole on part
 0), and the gated projection's EC steps run in the last part.  The shapes
@@ -32,9 +33,13 @@ def S():
 
 
 def k_parts(M, K, N, r, sms):
-    """The launch's rule: 128-token tiles (M < 512), projection tiles when r > 0."""
+    """The launch's rule: 256-token tiles only from M = 512 up and when they fill
+    at least half the SMs (no K parts then); else 128-token tiles, projection
+    tiles when r > 0, and the K parts."""
     if M >= 512:
-        return 1
+        mb256 = (M + 255) // 256
+        if 2 * ((mb256 if r else 0) + mb256 * (N // 256)) >= sms:
+            return 1
     mb = (M + 127) // 128
     ntiles = (mb if r else 0) + mb * (N // 256)
     kt = K // 64
@@ -53,6 +58,7 @@ CASES = [
     (128, 4096, 11008, 64, 0, 2),   # 44 tiles
     (64, 1024, 4096, 16, 0, 2),     # K = 1024: 16 k-steps, at most 2 parts
     (48, 4096, 4096, 0, 0, 8),      # no EC: 16 output tiles only
+    (512, 4096, 4096, 64, 0, 2),    # 34 tall tiles would fill too few SMs: 68 short ones x 2 parts
 ]
 
 

@@ -799,11 +799,16 @@ static int launch_tc_t(const TcPlan& p, const TcArgs& a, const CUtensorMap* maps
   return e == cudaSuccess ? SPEAR_OK : set_cuda_error("tc kernel launch", e);
 }
 
-// Tile height: 256 tokens from M = 512 up (twice the tensor-core work per
-// dequantised tile and per ring round trip), when the rank gate's parameters,
-// if any, fit beside three stages; 128 otherwise.
-static int tc_tile_rows(int M, const LayerView& L, bool with_ec) {
+// Tile height: 256 tokens (twice the tensor-core work per dequantised tile
+// and per ring round trip) once such tiles fill at least half the SMs, when
+// the rank gate's parameters, if any, fit beside three stages; 128 otherwise,
+// where K parts fill the SMs (at M = 512, N = 4096 the 34 tall tiles ran
+// their whole K on 34 SMs, as slow as M = 2048).
+static int tc_tile_rows(int M, const LayerView& L, bool with_ec, int sms) {
   if (M < 512) return 128;
+  const int mb = (M + 255) / 256;
+  const int tiles = (with_ec && L.r > 0 ? mb : 0) + mb * (L.N / TC_BN);
+  if (2 * tiles < sms) return 128;
   const bool rank = with_ec && L.r > 0 && L.gate_kind == 1;
   return (!rank || tc_smem(3, 256) + tc_gpar_bytes(L.gate_h, L.r) <= TC_SMEM_MAX) ? 256 : 128;
 }
@@ -812,7 +817,7 @@ int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
               WsHeader* hdr, int* mflags, int* kflags, float* kpart, __nv_bfloat16* gt, float* gate_out,
               int* mask_count, cudaStream_t st) {
   if (L.N % TC_BN) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "tensor-core path needs N %% 256 == 0 (N=%d)", L.N);
-  const int bmt = tc_tile_rows(M, L, with_ec);
+  const int bmt = tc_tile_rows(M, L, with_ec, p.grid);
   TcArgs a = {};
   a.scales = L.scales;
   a.y = y;
