@@ -242,6 +242,26 @@ int spear_read_status(void* ws, int* device_status, void* stream);
  * SPEAR_ERR_INVALID_ARG for another kernel value or wait_cycles < 1. */
 int spear_test_inject_timeout(int kernel, long long wait_cycles);
 
+/* ---- device-check build --------------------------------------------------
+ * The library can be built a second time with -DSPEAR_DEVICE_CHECKS
+ * (libspear_checked.so beside libspear.so): device-side bounds checks on the
+ * kernels' output stores (row < M, channels < N) and on their workspace
+ * partial slots, flags and published EC rows.  A failed check writes
+ * SPEAR_ERR_DEVICE_CHECK to the status word (spear_read_status), skips the
+ * access it guards and never traps; y is then unspecified.  In the normal
+ * build the checks compile away.
+ *
+ * spear_device_checks_enabled: 1 in the device-check build, 0 otherwise.
+ *
+ * spear_test_force_device_check (test hook): kernel 1 makes the decode
+ * kernel's output-store check fail, kernel 2 the tensor-core kernel's, in
+ * the launches that follow until called with 0 (process-wide).  The
+ * guarded stores are skipped, so no out-of-range access is ever made; the
+ * launch reports SPEAR_ERR_DEVICE_CHECK.  No effect in the normal build.
+ * SPEAR_ERR_INVALID_ARG for another kernel value. */
+int spear_device_checks_enabled(void);
+int spear_test_force_device_check(int kernel);
+
 /* ---- allocation-free decode call ---------------------------------------------
  * Not part of the method on the pages (they have no counterpart): an
  * interface for callers that cannot allocate device memory where they run

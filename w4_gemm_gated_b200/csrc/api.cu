@@ -1,6 +1,7 @@
 // C ABI of the library (declared in include/spear.h): argument validation,
 // workspace layout, the measured-time dispatch table and path selection.
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -35,6 +36,9 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 static std::mutex g_fault_mu;
 static TestFault g_fault = {0, 0};
+std::atomic<int> g_force_check{0};
+int test_force_check() { return g_force_check.load(); }
+
 TestFault test_fault() {
   std::lock_guard<std::mutex> lk(g_fault_mu);
   return g_fault;
@@ -153,7 +157,7 @@ static size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 // scratch after them (gated projection, K-split partials) grows with M.
 static constexpr int kMaxM = 65536;
 static constexpr int kFlagCap = kMaxM / 16 + 64;  // 16-token blocks (+ slack)
-static constexpr int kKFlagCap = 4 * 1024;         // K-part flags: 4 per (tile, part), tiles x parts <= SMs
+static constexpr int kKFlagCap = kKFlagCapacity;
 
 static WsLayout ws_layout_uncached(const LayerView& L, int M_max) {
   WsLayout w = {};
@@ -438,6 +442,21 @@ int spear_test_inject_timeout(int kernel, long long wait_cycles) {
   std::lock_guard<std::mutex> lk(g_fault_mu);
   g_fault = TestFault{kernel, kernel ? wait_cycles : 0};
   return SPEAR_OK;
+}
+
+int spear_test_force_device_check(int kernel) {
+  g_last_error.clear();
+  if (kernel < 0 || kernel > 2) return set_error(SPEAR_ERR_INVALID_ARG, "kernel=%d: must be 0, 1 or 2", kernel);
+  g_force_check.store(kernel);
+  return SPEAR_OK;
+}
+
+int spear_device_checks_enabled(void) {
+#ifdef SPEAR_DEVICE_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 size_t spear_w4_packed_bytes(int N, int K) {

@@ -51,6 +51,20 @@ __device__ __forceinline__ void st_release_gpu(int* p, int v) {
   asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Device-side argument checks of the debug build (-DSPEAR_DEVICE_CHECKS): a
+// failed check reports SPEAR_ERR_DEVICE_CHECK in the status word and the
+// access it guards is skipped; nothing traps or faults.  In the normal build
+// a check is `true` and its condition is not evaluated.
+#ifdef SPEAR_DEVICE_CHECKS
+__device__ __forceinline__ bool spear_dcheck(bool ok, WsHeader* h) {
+  if (!ok) report_status(h, SPEAR_ERR_DEVICE_CHECK);
+  return ok;
+}
+#define SPEAR_DCHECK(cond, hdr) ::spear::spear_dcheck((cond), (hdr))
+#else
+#define SPEAR_DCHECK(cond, hdr) true
+#endif
+
 // Spin until the n flags f[0..n) all equal want, their loads in flight
 // together (one round trip per poll), then an acquire fence; false (and a
 // status report) if the bound expires.

@@ -369,7 +369,7 @@ __device__ void decode_store_pair(const DecodeArgs& a, int pair, int lane, bool 
   __syncwarp();
   for (int idx = lane; idx < MT * 4; idx += 32) {
     const int m = idx >> 2, part = idx & 3;
-    if (m < a.M) {
+    if (m < a.M && SPEAR_DCHECK(32 * pair + 32 <= a.N, a.hdr)) {
       uint4 v = *reinterpret_cast<const uint4*>(stage + m * 32 + part * 8);
       uint4* dst = reinterpret_cast<uint4*>(a.y + (size_t)m * a.N + 32 * pair + part * 8);
       if (a.ec_only) {

@@ -300,7 +300,7 @@ __device__ void d2_store_strip(const D2Args& a, int p, float (&acc)[MT / 8][4], 
   }
   __syncwarp();
   const int m = lane >> 1, h = lane & 1;
-  if (m < a.M) {
+  if (m < a.M && SPEAR_DCHECK(16 * p + 16 <= a.N, a.hdr)) {
     uint4 v = *reinterpret_cast<const uint4*>(stage + m * 16 + 8 * h);
     uint4* dst = reinterpret_cast<uint4*>(a.y + (size_t)m * a.N + 16 * p + 8 * h);
     if (a.ec_only) {

@@ -72,6 +72,7 @@ struct D3Args {
   int own_cap;              // weight strips of the fullest CTA
   int tag_skew;             // test injection: publication flags are awaited at tag + skew (0 normally)
   long long pub_wait;       // bound of that wait (SM cycles)
+  int dcheck_force;         // test hook: the y-store check fails (device-check build)
   const uint8_t* pf[3];     // the next call's buffers to warm in L2 (prefetch_next hint)
   unsigned long long pf_bytes[3];
   short4 tab[D3_MAXCTA];    // per CTA: EC item (-1 none), first weight strip, weight strips, 0
@@ -547,7 +548,7 @@ __device__ __noinline__ void d3_finish_strip(const D3Args& a, uint8_t* sm, int j
   }
   __syncwarp();
   const int m = lane >> 1, hh = lane & 1;
-  if (m < a.M) {
+  if (m < a.M && SPEAR_DCHECK(16 * p + 16 <= a.N && !a.dcheck_force, a.hdr)) {
     uint4 v = *reinterpret_cast<const uint4*>(stage + m * 16 + 8 * hh);
     uint4* dst = reinterpret_cast<uint4*>(a.y + (size_t)m * a.N + 16 * p + 8 * hh);
     if (a.ec_only) {
@@ -820,7 +821,7 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
     int last = 0;
     if (lane == 0) last = atom_add_acqrel_cta(&s_eccnt, 1) == D3_NW - 1 ? 1 : 0;
     last = __shfl_sync(FULL, last, 0);
-    if (last && ok) {
+    if (last && ok && SPEAR_DCHECK(ec_item < D3_MAXE, a.hdr)) {
       float* dst = a.tf + (size_t)ec_item * MT * 16;
       if (ec_item < a.ES) {
         float tot[NT][4];
@@ -1169,6 +1170,7 @@ int launch_decode3(const LayerView& Lv, const __nv_bfloat16* x, int M, __nv_bflo
   const TestFault tf_ = test_fault();
   a.tag_skew = tf_.kernel == 1 ? 1 : 0;
   a.pub_wait = tf_.kernel == 1 ? tf_.cycles : kWaitCycles;
+  a.dcheck_force = test_force_check() == 1;
   for (int i = 0; i < 3; ++i) {
     a.pf[i] = static_cast<const uint8_t*>(Lv.pf[i]);
     a.pf_bytes[i] = Lv.pf_bytes[i];

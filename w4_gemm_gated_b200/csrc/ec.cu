@@ -336,7 +336,7 @@ __device__ void ec_item_update(const EcArgs& a, int item, int lane, __nv_bfloat1
   __syncwarp();
   for (int idx = lane; idx < 64 * 4; idx += 32) {
     const int m = idx >> 2, part = idx & 3;
-    if (m0 + m < a.M)
+    if (m0 + m < a.M && SPEAR_DCHECK(32 * pair + 32 <= a.N, a.hdr))
       *reinterpret_cast<uint4*>(a.y + (size_t)(m0 + m) * a.N + 32 * pair + part * 8) =
           *reinterpret_cast<const uint4*>(stage + m * 32 + part * 8);
   }

@@ -24,6 +24,11 @@ struct TestFault {
   long long cycles;
 };
 TestFault test_fault();
+// test hook: 1 forces the decode kernels' y-store check to fail, 2 the
+// tensor-core kernel's (device-check build only; 0 = off)
+int test_force_check();
+// K-part flags in the workspace: 4 per (tile, part, 128-row half), tiles x parts <= SMs
+constexpr int kKFlagCapacity = 4 * 1024;
 
 struct LayerView;
 // Validate a public layer description (same checks as every layer call).

@@ -87,6 +87,9 @@ struct TcArgs {
   int S;                  // K parts per tile (1: none); CTA b takes part b % S of tiles b / S, + grid / S, ...
   float* kpart;           // [tiles * S][4 warps][64][32 lanes][4] fp32 partial accumulators (S > 1)
   int* kflags;            // [tiles * S][4 * NH]: epoch + 1 once an epilogue warp's partial rows are out
+  int kpart_slots;        // 128 x 256 fp32 partial slots in the workspace (device-check build)
+  int kflag_cap;          // K-part flags in the workspace (device-check build)
+  int dcheck_force;       // test hook: the y-store check fails (device-check build)
 };
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -508,7 +511,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       bool run_gate = true;
       if (BMT == 128 && a.S > 1) {
         const int part = (int)(blockIdx.x % (unsigned)a.S);
-        const bool rows = ti.mb * BMT + h * TC_BM + q * 32 < a.M;
+        // (device-check build: this tile's partial slots and flags lie in the workspace)
+        const bool kp_ok =
+            SPEAR_DCHECK((tile + 1) * a.S <= a.kpart_slots && (tile + 1) * a.S * 4 * NH <= a.kflag_cap, a.hdr);
+        const bool rows = ti.mb * BMT + h * TC_BM + q * 32 < a.M && kp_ok;
         const int ncol = ti.kind == 0 ? a.NE : TC_BN;
         constexpr int QF = TC_BN * 32;  // floats of one warp's partial
         const float* qbase = a.kpart + ((size_t)tile * a.S * 4 * NH + 4 * h + q) * QF;
@@ -706,7 +712,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               v[i + 1] *= sc.y;
             }
           }
-          if (m < a.M) {
+          if (m < a.M && SPEAR_DCHECK(n0 + c0 + 32 <= a.N && !a.dcheck_force, a.hdr)) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
@@ -860,6 +866,9 @@ int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
   const TestFault tf_ = test_fault();
   a.tag_skew = tf_.kernel == 2 ? 1 : 0;
   a.pub_wait = tf_.kernel == 2 ? tf_.cycles : kWaitCycles;
+  a.kpart_slots = p.grid;  // the workspace holds one slot per SM
+  a.kflag_cap = kKFlagCapacity;
+  a.dcheck_force = test_force_check() == 2;
   CUtensorMap maps[5];
   memset(maps, 0, sizeof(maps));
   bool ok = tmap_2d_bf16(&maps[0], x, L.K, M, TC_BK, bmt) && tmap_packed_box(&maps[1], L.w, L.K, L.N, 1, TC_BN / 16);

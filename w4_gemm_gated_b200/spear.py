@@ -14,7 +14,10 @@ from dataclasses import dataclass
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspear.so")
+# SPEAR_DEVICE_CHECKS=1 loads the device-check build of the same library
+# (bounds checks that report SPEAR_ERR_DEVICE_CHECK; built beside it)
+_LIB_NAME = "libspear_checked.so" if os.environ.get("SPEAR_DEVICE_CHECKS") == "1" else "libspear.so"
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), _LIB_NAME)
 if not os.path.exists(_LIB_PATH):
     raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m w4_gemm_gated_b200.build`")
 _lib = ctypes.CDLL(_LIB_PATH)
@@ -85,6 +88,8 @@ EXPORTS = {
     "spear_linear_forward_decode_noalloc": (_i, ctypes.POINTER(LayerStruct), _vp, _i, _vp, _vp, _vp, _vp),
     "spear_read_status_noalloc": (_i, ctypes.POINTER(_i), _vp),
     "spear_test_inject_timeout": (_i, _i, ctypes.c_longlong),
+    "spear_device_checks_enabled": (_i,),
+    "spear_test_force_device_check": (_i, _i),
     "spear_dispatch_choice": (_i, ctypes.POINTER(LayerStruct), _i),
     "spear_dispatch_tune": (_i, ctypes.POINTER(LayerStruct), ctypes.POINTER(_i), _i, _vp, _vp, _vp, _sz, _vp, _sz,
                             _i, ctypes.POINTER(_f), _vp),
