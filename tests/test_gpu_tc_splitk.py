@@ -6,11 +6,14 @@ tiles are taken only where they fill at least half), the kernel splits every
 tile's K into S = 2, 4 or 8 parts (at least 8 k-steps each), one CTA per
 part.  Every part puts its fp32 accumulator in the workspace; each then sums,
 in part order, its 256 / S output channels (the projection tile whole on part
-0), and the gated projection's EC steps run in the last part.  The shapes
-below select each S (computed here with the launch's rule on this device's SM
-count and asserted), with the scalar gate, the pages' per-rank gate, no EC,
-group-128 scales, and token counts that leave the last 128-token block ragged
-or fill only its first 32-row quarter."""
+0), and the gated projection's EC steps run in the last part.  Where no split
+is taken but the tiles leave SMs idle, stream-K runs: every SM takes an equal
+run of the tiles' concatenated k-steps, and the CTA that holds a tile's first
+steps adds the other parts in k order and finishes it (with its EC steps).
+The shapes below select each S and stream-K (the schedule computed here with
+the launch's rule on this device's SM count and asserted), with the scalar
+gate, the pages' per-rank gate, no EC, group-128 scales, and token counts that
+leave the last 128-token block ragged or fill only its first 32-row quarter."""
 import numpy as np
 import pytest
 import torch
@@ -32,40 +35,52 @@ def S():
     return spear
 
 
-def k_parts(M, K, N, r, sms):
+def schedule(M, K, N, r, sms):
     """The launch's rule: 256-token tiles only from M = 512 up and when they fill
-    at least half the SMs (no K parts then); else 128-token tiles, projection
-    tiles when r > 0, and the K parts."""
+    at least half the SMs (persistent then); else 128-token tiles, projection
+    tiles when r > 0, K parts S = 2, 4, 8 while the tiles fill at most half
+    the SMs, and stream-K where no split was taken but tiles leave SMs idle.
+    Returns ("persistent", 1), ("split", S) or ("streamk", most parts of a tile)."""
     if M >= 512:
         mb256 = (M + 255) // 256
         if 2 * ((mb256 if r else 0) + mb256 * (N // 256)) >= sms:
-            return 1
+            return ("persistent", 1)
     mb = (M + 127) // 128
     ntiles = (mb if r else 0) + mb * (N // 256)
     kt = K // 64
     s = 1
     while s < 8 and ntiles * s * 2 <= sms and kt % (2 * s) == 0 and kt // (2 * s) >= 8:
         s *= 2
-    return s
+    if s > 1:
+        return ("split", s)
+    T = ntiles * kt
+    if ntiles < sms and T // sms >= 8:
+        lo = [c * T // sms for c in range(sms + 1)]
+        most = max(sum(1 for c in range(sms) if lo[c] < (t + 1) * kt and lo[c + 1] > t * kt) for t in range(ntiles))
+        return ("streamk", most)
+    return ("persistent", 1)
 
 
 CASES = [
-    # M, K, N, r, group, expected S
-    (32, 4096, 4096, 64, 0, 8),     # 17 tiles: one 32-row quarter of one token block
-    (100, 4096, 4096, 64, 128, 8),  # ragged token block, grouped scales
-    (256, 4096, 4096, 64, 0, 4),    # 34 tiles
-    (200, 4096, 4096, 32, 0, 4),    # two blocks, the second ragged
-    (128, 4096, 11008, 64, 0, 2),   # 44 tiles
-    (64, 1024, 4096, 16, 0, 2),     # K = 1024: 16 k-steps, at most 2 parts
-    (48, 4096, 4096, 0, 0, 8),      # no EC: 16 output tiles only
-    (512, 4096, 4096, 64, 0, 2),    # 34 tall tiles would fill too few SMs: 68 short ones x 2 parts
+    # M, K, N, r, group, expected schedule
+    (32, 4096, 4096, 64, 0, ("split", 8)),      # 17 tiles: one 32-row quarter of one token block
+    (100, 4096, 4096, 64, 128, ("split", 8)),   # ragged token block, grouped scales
+    (256, 4096, 4096, 64, 0, ("split", 4)),     # 34 tiles
+    (200, 4096, 4096, 32, 0, ("split", 4)),     # two blocks, the second ragged
+    (128, 4096, 11008, 64, 0, ("split", 2)),    # 44 tiles
+    (64, 1024, 4096, 16, 0, ("split", 2)),      # K = 1024: 16 k-steps, at most 2 parts
+    (48, 4096, 4096, 0, 0, ("split", 8)),       # no EC: 16 output tiles only
+    (512, 4096, 4096, 64, 0, ("split", 2)),     # 34 tall tiles would fill too few SMs: 68 short x 2
+    (256, 4096, 11008, 64, 0, ("streamk", 3)),  # 88 tiles: one run of ~38 k-steps per SM, a tile on up to 3
+    (384, 2048, 6144, 32, 0, ("streamk", 3)),   # 75 tiles of 32 k-steps, ~16 a CTA
+    (300, 4096, 8192, 64, 128, ("streamk", 3)), # ragged last block, grouped scales
 ]
 
 
-@pytest.mark.parametrize("M,K,N,r,group,S_want", CASES)
-def test_k_parts_match_oracle(S, M, K, N, r, group, S_want):
+@pytest.mark.parametrize("M,K,N,r,group,want", CASES)
+def test_k_parts_match_oracle(S, M, K, N, r, group, want):
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    assert k_parts(M, K, N, r, sms) == S_want
+    assert schedule(M, K, N, r, sms) == want
     L = synth.make_layer(M, K, N, r, b_g=-0.5, x_kind="t3", seed=1200 + M + r)
     layer = prepared(S, L, group)
     y, g, cnt, _ = run(S, layer, L.x, S.PATH_FUSED, gate=True)
@@ -77,7 +92,7 @@ def test_k_parts_match_oracle(S, M, K, N, r, group, S_want):
         assert int(cnt.item()) == int(np.sum(g_ref < 0.1))
 
 
-@pytest.mark.parametrize("M,N", [(32, 4096), (256, 4096)])
+@pytest.mark.parametrize("M,N", [(32, 4096), (256, 4096), (256, 11008)])
 def test_k_parts_rank_gate(S, M, N):
     # the per-rank gate (h = 16) on the projection tile's part 0, after the sum
     K, r, h = 4096, 64, 16

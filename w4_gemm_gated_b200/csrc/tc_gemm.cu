@@ -90,6 +90,8 @@ struct TcArgs {
   int kpart_slots;        // 128 x 256 fp32 partial slots in the workspace (device-check build)
   int kflag_cap;          // K-part flags in the workspace (device-check build)
   int dcheck_force;       // test hook: the y-store check fails (device-check build)
+  int sk;                 // 1: stream-K schedule (each CTA an equal run of the tiles' k-steps)
+  long long sk_T;         // stream-K: k-steps of all tiles (tiles x K / 64)
 };
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -167,30 +169,81 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 // schedule shared by all roles
 // ---------------------------------------------------------------------------
 struct TileInfo {
+  int tile;    // projection tiles first, then output tiles
   int kind;    // 0 = projection tile, 1 = output tile
   int mb, nb;
-  int k0, nk;  // this CTA's K part of the tile: k-steps k0 .. k0 + nk - 1
-  int steps;   // k-steps of this tile in this CTA (its K part, then the EC steps in the last part)
+  int k0, nk;  // this CTA's k-steps of the tile: k0 .. k0 + nk - 1
+  int steps;   // k-steps here: its part, then the EC steps where this CTA finishes the tile
+  int role;    // 0 whole tile; 1 K part `part` of S (column shares); 2 stream-K part sent to the
+               // tile's owner; 3 stream-K owner (the tile's first k-steps) of `part` parts
+  int part;
 };
 
-__device__ __forceinline__ TileInfo tile_info(const TcArgs& a, int tile) {
+// The units of work of this CTA, in the order every role takes them:
+//  - persistent (S == 1, no stream-K): tiles c, c + G, c + 2 G, ..., whole;
+//  - K parts (S > 1): one unit, K part c % S of tile c / S;
+//  - stream-K: the CTA's share [c T / G, (c + 1) T / G) of the T = tiles x K/64
+//    k-steps, tile by tile in order.  A tile begun in an earlier CTA is a part
+//    sent to that CTA (the tile's owner); a tile begun here is owned here and
+//    takes the parts of the CTAs that finish it.  A sent part is always the
+//    CTA's first unit and an owned tile with parts its last, so no wait cycles.
+__device__ __forceinline__ long long sk_lo(const TcArgs& a, int c) { return (long long)c * a.sk_T / gridDim.x; }
+
+__device__ __forceinline__ int unit_count(const TcArgs& a, int ntiles) {
+  const int c = (int)blockIdx.x, G = (int)gridDim.x;
+  if (a.sk) {
+    const long long KT = a.K / TC_BK, lo = sk_lo(a, c), hi = sk_lo(a, c + 1);
+    return hi > lo ? (int)((hi - 1) / KT - lo / KT) + 1 : 0;
+  }
+  if (a.S > 1) return 1;
+  return c < ntiles ? (ntiles - 1 - c) / G + 1 : 0;
+}
+
+__device__ __forceinline__ TileInfo unit_info(const TcArgs& a, int u) {
   TileInfo t;
   const int KT = a.K / TC_BK;
   const int nproj = a.with_ec ? a.Mb : 0;
-  const int part = (int)(blockIdx.x % (unsigned)a.S);
-  t.nk = KT / a.S;
-  t.k0 = part * t.nk;
-  if (tile < nproj) {
+  const int c = (int)blockIdx.x, G = (int)gridDim.x;
+  t.role = 0;
+  t.part = 0;
+  if (a.sk) {
+    const long long lo = sk_lo(a, c), hi = sk_lo(a, c + 1);
+    t.tile = (int)(lo / KT) + u;
+    const long long t0 = (long long)t.tile * KT;
+    const long long s0 = lo > t0 ? lo : t0, s1 = hi < t0 + KT ? hi : t0 + KT;
+    t.k0 = (int)(s0 - t0);
+    t.nk = (int)(s1 - s0);
+    if (t.k0 > 0) {
+      t.role = 2;
+    } else {
+      int np = 1;  // this CTA and the next ones that start inside the tile
+      while (c + np < G && sk_lo(a, c + np) < t0 + KT) ++np;
+      t.role = 3;
+      t.part = np;
+    }
+  } else if (a.S > 1) {
+    t.tile = c / a.S;
+    t.role = 1;
+    t.part = c % a.S;
+    t.nk = KT / a.S;
+    t.k0 = t.part * t.nk;
+  } else {
+    t.tile = c + u * G;
+    t.k0 = 0;
+    t.nk = KT;
+  }
+  const bool finishes = t.role == 0 || t.role == 3 || (t.role == 1 && t.part == a.S - 1);
+  if (t.tile < nproj) {
     t.kind = 0;
-    t.mb = tile;
+    t.mb = t.tile;
     t.nb = 0;
     t.steps = t.nk;
   } else {
-    const int i = tile - nproj;
+    const int i = t.tile - nproj;
     t.kind = 1;
     t.mb = i / a.Nb;
     t.nb = i % a.Nb;
-    t.steps = t.nk + (a.with_ec && part == a.S - 1 ? a.ec_steps : 0);
+    t.steps = t.nk + (a.with_ec && finishes ? a.ec_steps : 0);
   }
   return t;
 }
@@ -283,8 +336,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int epoch = *reinterpret_cast<volatile int*>(&a.hdr->epoch);
   const int ntiles = (a.with_ec ? a.Mb : 0) + a.Mb * a.Nb;
-  // tiles of this CTA: groups of S consecutive CTAs share each tile's K parts
-  const int t_first = (int)blockIdx.x / a.S, t_step = (int)gridDim.x / a.S;
+  const int nunits = unit_count(a, ntiles);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -322,8 +374,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t ph = 0;
       int issued = 0;  // stages whose loads went out
       bool ok = true;
-      for (int tile = t_first; tile < ntiles && ok; tile += t_step) {
-        const TileInfo ti = tile_info(a, tile);
+      for (int u = 0; u < nunits && ok; ++u) {
+        const TileInfo ti = unit_info(a, u);
         for (int k = 0; k < ti.steps && ok; ++k) {
           ok = mbar_wait(&empty[s], ph ^ 1, abort_flag, a.hdr);
           if (!ok) break;
@@ -356,9 +408,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                   tma_prefetch_2d(&tm_bpt, e * TC_BK, ti.nb * TC_BN);
                   tma_prefetch_2d(&tm_gt, e * TC_BK, ti.mb * BMT);
                 }
-              const int nt = tile + t_step;
-              if (nt < ntiles) {
-                const TileInfo tn = tile_info(a, nt);
+              if (u + 1 < nunits) {
+                const TileInfo tn = unit_info(a, u + 1);
                 if (tn.kind == 1 && j < tn.nk) {
                   tma_prefetch_2d(&tm_x, (tn.k0 + j) * TC_BK, tn.mb * BMT);
                   tma_prefetch_3d(&tm_w, 0, tn.k0 + j, tn.nb * (TC_BN / 16));
@@ -368,7 +419,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             // the CTA's first tile: once the ring's first loads are out, warm the
             // steps after them that the per-step warm-up above does not reach
             // (later tiles had theirs warmed during the previous tile's tail)
-            if (tile == t_first && k == min(NST, ti.nk) - 1)
+            if (u == 0 && k == min(NST, ti.nk) - 1)
               for (int pk = NST; pk < TC_PREFETCH && pk < ti.nk; ++pk) {
                 tma_prefetch_2d(&tm_x, (ti.k0 + pk) * TC_BK, ti.mb * BMT);
                 tma_prefetch_3d(&tm_w, 0, ti.k0 + pk, ti.nb * (TC_BN / 16));
@@ -417,8 +468,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       int last_s = -1;      // stage (and its phase) of the last commit
       uint32_t last_ph = 0;
       bool ok = true;
-      for (int tile = t_first; tile < ntiles && ok; tile += t_step) {
-        const TileInfo ti = tile_info(a, tile);
+      for (int u = 0; u < nunits && ok; ++u) {
+        const TileInfo ti = unit_info(a, u);
         ok = mbar_wait(&acc_empty[buf], aph[buf] ^ 1, abort_flag, a.hdr);
         if (!ok) break;
         tc_fence_after();
@@ -478,8 +529,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     int buf = 0;
     uint32_t aph[2] = {0, 0};
     bool ok = true;
-    for (int tile = t_first; tile < ntiles && ok; tile += t_step) {
-      const TileInfo ti = tile_info(a, tile);
+    for (int u = 0; u < nunits && ok; ++u) {
+      const TileInfo ti = unit_info(a, u);
+      const int tile = ti.tile;
       ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], aph[buf], abort_flag, a.hdr));
       if (!ok) break;
       tc_fence_after();
@@ -508,9 +560,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       // holds one tile when S > 1).  A warp whose 32 rows are all past M skips
       // the exchange on every part alike.
       int lo = 0, hi = TC_BN;
-      bool run_gate = true;
-      if (BMT == 128 && a.S > 1) {
-        const int part = (int)(blockIdx.x % (unsigned)a.S);
+      bool run_gate = true, sent = false;
+      if (BMT == 128 && ti.role == 1) {
+        const int part = ti.part;
         // (device-check build: this tile's partial slots and flags lie in the workspace)
         const bool kp_ok =
             SPEAR_DCHECK((tile + 1) * a.S <= a.kpart_slots && (tile + 1) * a.S * 4 * NH <= a.kflag_cap, a.hdr);
@@ -610,7 +662,107 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
         }
       }
-      if (ti.kind == 0 && !run_gate) {
+      // stream-K: a sent part puts its accumulator in the workspace slot of this
+      // CTA ([column/4][lane][4] per warp, as above) and raises its flag; the
+      // owner waits for the parts of the CTAs after it, reads them with one
+      // bulk copy per part and chunk into the ring (idle: an owned tile with
+      // parts is the CTA's last unit), and adds them in k order to its own
+      // accumulator, on which the epilogue below then runs.
+      if (BMT == 128 && (ti.role == 2 || (ti.role == 3 && ti.part > 1))) {
+        constexpr int QF = TC_BN * 32;
+        const bool rows = ti.mb * BMT + h * TC_BM + q * 32 < a.M &&
+                          SPEAR_DCHECK((int)gridDim.x <= a.kpart_slots && (int)gridDim.x * 4 * NH <= a.kflag_cap,
+                                       a.hdr);
+        const int ncol = ti.kind == 0 ? a.NE : TC_BN;
+        auto slot = [&](int cta) { return a.kpart + ((size_t)cta * 4 * NH + 4 * h + q) * QF; };
+        auto sflag = [&](int cta) { return a.kflags + cta * 4 * NH + 4 * h + q; };
+        if (ti.role == 2) {
+          sent = true;
+          if (rows) {
+            float4* pdst = reinterpret_cast<float4*>(slot((int)blockIdx.x));
+            for (int c0 = 0; c0 < ncol; c0 += 16) {
+              float v[16];
+              tmem_ld16(taddr + c0, v);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                pdst[(c0 / 4 + i) * 32 + lane] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
+            // the warp barrier orders every lane's stores before lane 0's release
+            __syncwarp();
+            if (lane == 0) st_release_gpu(sflag((int)blockIdx.x), epoch + 1);
+          }
+        } else if (rows) {
+          const int nother = ti.part - 1;  // parts of CTAs blockIdx.x + 1 .. + nother
+          const int nw = min(4, (a.M - ti.mb * BMT - h * TC_BM + 31) / 32);
+          const int XW = (NST * tc_stage_bytes(BMT) / nw) & ~1023;
+          uint8_t* xw = smem + q * XW;
+          uint64_t* xbar = reinterpret_cast<uint64_t*>(xw + XW - 128);
+          int CC = ncol;
+          while (nother * CC * 128 > XW - 128) CC = (CC / 2 + 15) & ~15;
+          const int CB = nother * CC * 128;
+          const int nch = (ncol + CC - 1) / CC;
+          const int NB = min(min(nch, (XW - 128) / CB), 16);
+          if (lane == 0) {
+            for (int b = 0; b < NB; ++b) mbar_init(&xbar[b], 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+          }
+          const bool fok = lane >= nother || wait_flag_eq(sflag((int)blockIdx.x + 1 + lane), epoch + 1, a.hdr);
+          if (!__all_sync(0xffffffffu, fok)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          auto issue = [&](int ch) {  // lane 0: columns CC ch .. of every other part
+            const int b = ch % NB, c0 = ch * CC, nb = (min(ncol, c0 + CC) - c0) * 128;
+            mbar_arrive_tx(&xbar[b], nother * nb);
+            for (int pp = 0; pp < nother; ++pp)
+              bulk_g2s(xw + b * CB + pp * CC * 128, slot((int)blockIdx.x + 1 + pp) + c0 * 32, nb, &xbar[b]);
+          };
+          __syncwarp();
+          if (lane == 0) {
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            for (int ch = 0; ch < NB; ++ch) issue(ch);
+          }
+          int ch = 0;
+          for (; ch < nch; ++ch) {
+            const int b = ch % NB, c0 = ch * CC, c1 = min(ncol, c0 + CC);
+            if (!__all_sync(0xffffffffu, mbar_wait(&xbar[b], (ch / NB) & 1, abort_flag, a.hdr))) break;
+            for (int g = c0; g < c1; g += 16) {
+              float sum[16];
+              tmem_ld16(taddr + g, sum);  // this CTA's part comes first in k order
+              for (int pp = 0; pp < nother; ++pp) {
+                const float4* src = reinterpret_cast<const float4*>(xw + b * CB + pp * CC * 128 + (g - c0) * 128) + lane;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float4 v = src[32 * i];
+                  sum[4 * i] += v.x;
+                  sum[4 * i + 1] += v.y;
+                  sum[4 * i + 2] += v.z;
+                  sum[4 * i + 3] += v.w;
+                }
+              }
+              tmem_st16(taddr + g, sum);
+            }
+            __syncwarp();
+            if (lane == 0 && ch + NB < nch) {
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+              issue(ch + NB);
+            }
+          }
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+          if (ch < nch) {
+            // gave up: let the copies in flight land before the ring is released
+            if (lane == 0)
+              for (int c = ch; c < nch && c < ch + NB; ++c) tc_drain(&xbar[c % NB], (c / NB) & 1);
+            __syncwarp();
+            ok = false;
+            break;
+          }
+        }
+      }
+      if (sent) {
+        // the tile's owner stores it
+      } else if (ti.kind == 0 && !run_gate) {
         // another part runs this projection tile's gate
       } else if (ti.kind == 0) {
         // projection tile: columns 0..r-1 = t, column r = gate logit
@@ -735,8 +887,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (int tile = t_first; tile < ntiles && ok; tile += t_step) {
-      const TileInfo ti = tile_info(a, tile);
+    for (int u = 0; u < nunits && ok; ++u) {
+      const TileInfo ti = unit_info(a, u);
       for (int k = 0; k < ti.steps && ok; ++k) {
         ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, a.hdr));
         if (!ok) break;
@@ -798,7 +950,7 @@ static int launch_tc_t(const TcPlan& p, const TcArgs& a, const CUtensorMap* maps
   if (attr_err != cudaSuccess) return set_cuda_error("cudaFuncSetAttribute(tc)", attr_err);
   const int ntiles = (a.with_ec ? a.Mb : 0) + a.Mb * a.Nb;
   const int groups = ntiles < p.grid / a.S ? ntiles : p.grid / a.S;
-  const int grid = groups * a.S;
+  const int grid = a.sk ? p.grid : groups * a.S;
   const size_t smem = tc_smem(a.nst, BMT) + (a.gate_kind == 1 ? tc_gpar_bytes(a.gate_h, a.r) : 0);
   tc_kernel<GROUP, BMT><<<grid, TC_THREADS, smem, st>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4]);
   cudaError_t e = cudaGetLastError();
@@ -862,6 +1014,14 @@ int launch_tc(const TcPlan& p, const LayerView& L, const __nv_bfloat16* x, int M
     const int ntiles = (a.with_ec ? a.Mb : 0) + a.Mb * a.Nb;
     const int KT = L.K / TC_BK;
     while (a.S < 8 && ntiles * a.S * 2 <= p.grid && KT % (a.S * 2) == 0 && KT / (a.S * 2) >= 8) a.S *= 2;
+    // stream-K where the tiles leave SMs idle but no K split was taken (more
+    // than half as many tiles as SMs, or a K that the split cannot divide):
+    // every SM takes an equal run of at least 8 of the tiles' k-steps
+    const long long T = (long long)ntiles * KT;
+    if (a.S == 1 && ntiles < p.grid && T / p.grid >= 8) {
+      a.sk = 1;
+      a.sk_T = T;
+    }
   }
   const TestFault tf_ = test_fault();
   a.tag_skew = tf_.kernel == 2 ? 1 : 0;
