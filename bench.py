@@ -157,8 +157,8 @@ def time_oracle(target_s: float = 15.0, n_cols: int = 1376):
 # DRAM bytes per decode launch from the ncu captures summarised in profiles/
 # (dram__bytes_read.sum + dram__bytes_write.sum, one launch at M = 1 and at M = 16),
 # valid only while the decode kernel sources are the ones captured.
-DECODE_TRAFFIC = {"sources_sha1": "aa757fd427da2db92983e161edde880fa1e9e292",
-                  "bytes_per_launch": {1: 24588800, 16: 24722176}}
+DECODE_TRAFFIC = {"sources_sha1": "2b2f809a8cf32a5360f470a3cd29ed42a7616859",
+                  "bytes_per_launch": {1: 24592384, 16: 24724992}}
 DECODE_SOURCES = ("w4_gemm_gated_b200/csrc/decode3.cu", "w4_gemm_gated_b200/csrc/common.cuh",
                   "w4_gemm_gated_b200/csrc/tma.cuh")
 

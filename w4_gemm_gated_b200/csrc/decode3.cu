@@ -243,6 +243,58 @@ __device__ __forceinline__ void d3_ecterm(const __nv_bfloat16* bp, const __nv_bf
   }
 }
 
+// The same with the scalar gate, gt formed by the warp itself from t and the
+// gate logit in shared memory (ts [MT][r], logits at ts[MT r + m]): the words
+// it would have read from gt, bf16(g t) with g = sigmoid(logit + b_g), zero
+// for padded tokens, in the same arithmetic as the gt builder.
+template <int MT, int S, int NCH>
+__device__ __forceinline__ void d3_ecterm_scalar(const __nv_bfloat16* bp, const float* ts, int M, float b_g, int r,
+                                                 int lane, float (&acc)[MT / 8][4]) {
+  constexpr int NT = MT / 8;
+  const int rho = lane >> 2, c = lane & 3;
+  float g[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int m = nt * 8 + rho;
+    g[nt] = m < M ? sigmoidf_(ts[MT * r + m] + b_g) : 0.f;
+  }
+#pragma unroll
+  for (int ch = 0; ch < NCH; ++ch) {
+    uint32_t b0[8], b1[8], gw[NT][8];
+    d3_lds_words<S>(bp + rho * r + 64 * ch + 4 * S * c, b0);
+    d3_lds_words<S>(bp + (rho + 8) * r + 64 * ch + 4 * S * c, b1);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int m = nt * 8 + rho;
+      const float2* tv = reinterpret_cast<const float2*>(ts + m * r + 64 * ch + 4 * S * c);
+#pragma unroll
+      for (int i = 0; i < 2 * S; ++i) {
+        const float2 t2 = tv[i];
+        gw[nt][i] = m < M ? pack_bf16x2(g[nt] * t2.x, g[nt] * t2.y) : 0u;
+      }
+    }
+#pragma unroll
+    for (int s2 = 0; s2 < S; ++s2) {
+      const uint32_t af[4] = {b0[2 * s2], b1[2 * s2], b0[2 * s2 + 1], b1[2 * s2 + 1]};
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc[nt], af, gw[nt][2 * s2], gw[nt][2 * s2 + 1]);
+    }
+  }
+}
+
+template <int MT>
+__device__ __forceinline__ void d3_ecterm_scalar_r(const __nv_bfloat16* bp, const float* ts, int M, float b_g, int r,
+                                                   int lane, float (&acc)[MT / 8][4]) {
+  if (r == 16)
+    d3_ecterm_scalar<MT, 1, 1>(bp, ts, M, b_g, r, lane, acc);
+  else if (r == 32)
+    d3_ecterm_scalar<MT, 2, 1>(bp, ts, M, b_g, r, lane, acc);
+  else if (r == 64)
+    d3_ecterm_scalar<MT, 4, 1>(bp, ts, M, b_g, r, lane, acc);
+  else
+    d3_ecterm_scalar<MT, 4, 2>(bp, ts, M, b_g, r, lane, acc);
+}
+
 template <int MT>
 __device__ __forceinline__ void d3_ecterm_r(const __nv_bfloat16* bp, const __nv_bfloat16* gts, int r, int lane,
                                             float (&acc)[MT / 8][4]) {
@@ -531,7 +583,13 @@ __device__ __noinline__ void d3_finish_strip(const D3Args& a, uint8_t* sm, int j
         tot[nt][3] += v.w;
       }
   }
-  if (a.ES > 0) d3_ecterm_r<MT>(bps + (size_t)j * 16 * a.r, gts, a.r, lane, tot);
+  if (a.ES > 0) {
+    if (a.gate_kind == 0)
+      d3_ecterm_scalar_r<MT>(bps + (size_t)j * 16 * a.r, reinterpret_cast<const float*>(sm + SL.ts), a.M, a.b_g, a.r,
+                             lane, tot);
+    else
+      d3_ecterm_r<MT>(bps + (size_t)j * 16 * a.r, gts, a.r, lane, tot);
+  }
   float s0 = 1.f, s1 = 1.f;
   if (!GROUP) {
     s0 = __half2float(scs[j * 16 + rho]);
@@ -910,10 +968,11 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
     }
   }
   if (fetcher && s_fetched) ok = __all_sync(FULL, d3_wait(tsbar, 0, abortp, a.hdr));
-  if (fetcher && ok && a.gate_kind == 0) {
-    // scalar gate, by this warp alone: g = sigmoid(logit + b_g) and
-    // gt = bf16(g t) for the live tokens (zero rows for the padded ones);
-    // the strip warps wait on gtbar, not on the whole CTA
+  if (fetcher && ok && a.gate_kind == 0 && blockIdx.x == 0) {
+    // scalar gate, CTA 0 only, which reports the gates: g = sigmoid(logit +
+    // b_g) and gt = bf16(g t) for the live tokens (zero rows for the padded
+    // ones).  The strip warps form their own gt words from t once it has
+    // landed (they wait on tsbar), so no CTA waits for this warp.
     const int gs = a.r + 8, half = a.r / 2;
     if (lane < MT) gv[lane] = lane < a.M ? sigmoidf_(ts[MT * a.r + lane] + a.b_g) : 0.f;
     __syncwarp();
@@ -949,7 +1008,7 @@ __global__ void __launch_bounds__(D3_THREADS, 1)
     bool eok = n_w > warp ? __all_sync(FULL, d3_wait(epibar, 0, abortp, a.hdr)) : false;
     for (int j = warp; j < n_w && eok; j += D3_NW) {
       if (!a.ec_only) eok = __all_sync(FULL, d3_wait(&pbar[n_ecu + j], 0, abortp, a.hdr));
-      if (eok && has_ec && a.gate_kind == 0) eok = __all_sync(FULL, d3_wait(gtbar, 0, abortp, a.hdr));
+      if (eok && has_ec && a.gate_kind == 0) eok = __all_sync(FULL, d3_wait(tsbar, 0, abortp, a.hdr));
       if (eok) d3_finish_strip<MT, GROUP>(a, sm, j, w_lo + j, ubase(n_ecu + j), CH, lane, warp);
     }
   }
