@@ -378,3 +378,28 @@ def test_binding_prototypes_match_the_header(S):
         got = [_ctypes_kind(t) for t in sig[1:]]
         assert got == want, (name, got, want)
         assert _ctypes_kind(sig[0]) == ret_kind, (name, sig[0], ret)
+
+
+def test_device_check_build_hooks(S):
+    # the normal build reports its checks off; the forced-check hook validates
+    # its argument (it has no effect here: no launch runs)
+    assert S.F["spear_device_checks_enabled"]() == 0
+    assert S.F["spear_test_force_device_check"](3) == S.ERR_INVALID_ARG
+    assert S.F["spear_test_force_device_check"](-1) == S.ERR_INVALID_ARG
+    assert S.F["spear_test_force_device_check"](0) == S.OK
+
+
+def test_device_check_build_loads_with_its_variable(S):
+    # SPEAR_DEVICE_CHECKS=1 makes the binding load the device-check build,
+    # which exports the same symbols and reports its checks on
+    import subprocess
+    import sys
+    from w4_gemm_gated_b200 import build
+    build.build(checked=True)
+    code = ("from w4_gemm_gated_b200 import spear as S; "
+            "print(S.LIB_PATH.endswith('libspear_checked.so'), S.F['spear_device_checks_enabled']())")
+    env = dict(os.environ, SPEAR_DEVICE_CHECKS="1", PYTHONPATH=ROOT)
+    out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True,
+                         timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert out.stdout.split() == ["True", "1"]
