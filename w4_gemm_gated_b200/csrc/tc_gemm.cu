@@ -23,6 +23,12 @@
 // same accumulator (B' = B / s_n is folded once per layer, so s_n applies
 // to the sum), so the EC costs neither a second kernel nor a pass over y.
 //
+// Schedules (a CTA per SM): with enough tiles, a persistent loop over whole
+// tiles; while the tiles fill at most half the SMs, each tile's K split into
+// S = 2, 4 or 8 parts whose fp32 partials each part sums for a 256/S-channel
+// share; in between, stream-K, each SM an equal run of the tiles' k-steps,
+// a tile finished by the CTA that holds its first k-steps (unit_info).
+//
 // Every wait on an mbarrier or a flag is bounded; on expiry the kernel
 // records SPEAR_ERR_TIMEOUT and all roles leave their loops.
 #include <cuda.h>
