@@ -260,6 +260,17 @@ int spear_test_inject_timeout(int kernel, long long wait_cycles);
  * launch reports SPEAR_ERR_DEVICE_CHECK.  No effect in the normal build.
  * SPEAR_ERR_INVALID_ARG for another kernel value. */
 int spear_device_checks_enabled(void);
+
+/* ---- tracing ---------------------------------------------------------------
+ * NVTX ranges named for the call around the layer calls, the preparation
+ * calls, the workspace and status calls and the dispatcher's tuning, for a
+ * profiler's timeline (ncu --nvtx, or any NVTX tool).  Off by default; on
+ * when the environment holds SPEAR_NVTX=1 at the first call, or after
+ * spear_set_tracing(1).  With no tool attached a range costs a branch.
+ * spear_set_tracing: on != 0 turns it on, 0 off (process-wide); SPEAR_OK.
+ * spear_tracing_enabled: 1 when on. */
+int spear_set_tracing(int on);
+int spear_tracing_enabled(void);
 int spear_test_force_device_check(int kernel);
 
 /* ---- allocation-free decode call ---------------------------------------------

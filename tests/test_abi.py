@@ -403,3 +403,17 @@ def test_device_check_build_loads_with_its_variable(S):
                          timeout=300)
     assert out.returncode == 0, out.stderr[-2000:]
     assert out.stdout.split() == ["True", "1"]
+
+
+def test_tracing_switch(S):
+    # NVTX ranges around the calls: off unless asked; a call traced with no
+    # tool attached (and no GPU needed: it fails validation) still behaves
+    assert S.F["spear_tracing_enabled"]() == (1 if os.environ.get("SPEAR_NVTX") == "1" else 0)
+    try:
+        assert S.F["spear_set_tracing"](1) == S.OK
+        assert S.F["spear_tracing_enabled"]() == 1
+        assert S.F["spear_w4_pack"](None, 16, 64, None, None) == S.ERR_INVALID_ARG
+        assert S.F["spear_workspace_init"](None, 0, None) == S.ERR_INVALID_ARG
+    finally:
+        S.F["spear_set_tracing"](0)
+    assert S.F["spear_tracing_enabled"]() == 0

@@ -3,6 +3,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <map>
@@ -10,6 +11,8 @@
 #include <string>
 #include <tuple>
 #include <vector>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -37,6 +40,26 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 static std::mutex g_fault_mu;
 static TestFault g_fault = {0, 0};
 std::atomic<int> g_force_check{0};
+
+// tracing: -1 until the environment is read (SPEAR_NVTX=1 turns it on)
+static std::atomic<int> g_trace{-1};
+static bool tracing() {
+  int v = g_trace.load();
+  if (v < 0) {
+    const char* e = std::getenv("SPEAR_NVTX");
+    int expected = -1;
+    g_trace.compare_exchange_strong(expected, (e && e[0] == '1') ? 1 : 0);
+    v = g_trace.load();
+  }
+  return v > 0;
+}
+TraceRange::TraceRange(const char* name) : on(tracing()) {
+  if (on) nvtxRangePushA(name);
+}
+TraceRange::~TraceRange() {
+  if (on) nvtxRangePop();
+}
+void set_tracing(bool on) { g_trace.store(on ? 1 : 0); }
 int test_force_check() { return g_force_check.load(); }
 
 TestFault test_fault() {
@@ -451,6 +474,14 @@ int spear_test_force_device_check(int kernel) {
   return SPEAR_OK;
 }
 
+int spear_set_tracing(int on) {
+  g_last_error.clear();
+  set_tracing(on != 0);
+  return SPEAR_OK;
+}
+
+int spear_tracing_enabled(void) { return tracing() ? 1 : 0; }
+
 int spear_device_checks_enabled(void) {
 #ifdef SPEAR_DEVICE_CHECKS
   return 1;
@@ -472,6 +503,7 @@ size_t spear_scale_count(int N, int K, int group) {
 }
 
 int spear_w4_quantize(const float* W, int K, int N, int group, int8_t* q, uint16_t* scales, void* stream) {
+  TraceRange trace_("spear_w4_quantize");
   g_last_error.clear();
   if (!W || !q || !scales) return set_error(SPEAR_ERR_INVALID_ARG, "NULL pointer");
   if (K <= 0 || N <= 0 || K % 32 || N % 32)
@@ -483,6 +515,7 @@ int spear_w4_quantize(const float* W, int K, int N, int group, int8_t* q, uint16
 }
 
 int spear_w4_pack(const int8_t* q, int N, int K, uint8_t* packed, void* stream) {
+  TraceRange trace_("spear_w4_pack");
   g_last_error.clear();
   if (!q || !packed) return set_error(SPEAR_ERR_INVALID_ARG, "NULL pointer");
   if (N <= 0 || K <= 0 || N % 16 || K % 64)
@@ -492,6 +525,7 @@ int spear_w4_pack(const int8_t* q, int N, int K, uint8_t* packed, void* stream) 
 }
 
 int spear_w4_unpack(const uint8_t* packed, int N, int K, int8_t* q, void* stream) {
+  TraceRange trace_("spear_w4_unpack");
   g_last_error.clear();
   if (!q || !packed) return set_error(SPEAR_ERR_INVALID_ARG, "NULL pointer");
   if (N <= 0 || K <= 0 || N % 16 || K % 64)
@@ -501,6 +535,7 @@ int spear_w4_unpack(const uint8_t* packed, int N, int K, int8_t* q, void* stream
 }
 
 int spear_ec_prescale_B(const uint16_t* B, const uint16_t* scales, int r, int N, uint16_t* Bp, void* stream) {
+  TraceRange trace_("spear_ec_prescale_B");
   g_last_error.clear();
   if (!B || !scales || !Bp) return set_error(SPEAR_ERR_INVALID_ARG, "NULL pointer");
   if (r <= 0 || N <= 0) return set_error(SPEAR_ERR_UNSUPPORTED_SHAPE, "r and N must be positive");
@@ -514,6 +549,7 @@ size_t spear_ec_bpt_count(int N, int r) { return (N > 0 && r > 0) ? (size_t)N * 
 
 int spear_ec_pack(const uint16_t* A, const uint16_t* B, const uint16_t* w_g, const uint16_t* scales, int K, int N,
                   int r, int group, uint16_t* AgT, uint16_t* BpT, void* stream) {
+  TraceRange trace_("spear_ec_pack");
   g_last_error.clear();
   if (!A || !B || !w_g || !AgT || !BpT || (group == 0 && !scales)) return set_error(SPEAR_ERR_INVALID_ARG, "NULL pointer");
   int rc = check_kn(K, N);
@@ -539,6 +575,7 @@ size_t spear_workspace_bytes(const spear_layer* layer, int M_max) {
 }
 
 int spear_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  TraceRange trace_("spear_workspace_init");
   g_last_error.clear();
   if (!ws || ws_bytes < kWsHeaderBytes) return set_error(SPEAR_ERR_INVALID_ARG, "bad workspace");
   cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
@@ -547,17 +584,20 @@ int spear_workspace_init(void* ws, size_t ws_bytes, void* stream) {
 
 int spear_linear_forward(const spear_layer* layer, const uint16_t* x, int M, uint16_t* y, void* ws, size_t ws_bytes,
                          float* gate_out, int* mask_count, void* stream) {
+  TraceRange trace_("spear_linear_forward");
   g_last_error.clear();
   return forward_impl(layer, x, M, y, ws, ws_bytes, gate_out, mask_count, SPEAR_PATH_AUTO, stream);
 }
 
 int spear_linear_forward_path(const spear_layer* layer, const uint16_t* x, int M, uint16_t* y, void* ws,
                               size_t ws_bytes, float* gate_out, int* mask_count, int path, void* stream) {
+  TraceRange trace_("spear_linear_forward_path");
   g_last_error.clear();
   return forward_impl(layer, x, M, y, ws, ws_bytes, gate_out, mask_count, path, stream);
 }
 
 int spear_read_status(void* ws, int* device_status, void* stream) {
+  TraceRange trace_("spear_read_status");
   g_last_error.clear();
   if (!ws || !device_status) return set_error(SPEAR_ERR_INVALID_ARG, "NULL pointer");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -761,6 +801,7 @@ int spear_dispatch_load(const char* path) {
 
 int spear_dispatch_tune(const spear_layer* layer, const int* Ms, int nM, const uint16_t* x, uint16_t* y, void* ws,
                         size_t ws_bytes, void* flush, size_t flush_bytes, int reps, float* times_us, void* stream) {
+  TraceRange trace_("spear_dispatch_tune");
   g_last_error.clear();
   LayerView L;
   int rc = check_layer(layer, &L);

@@ -27,6 +27,15 @@ TestFault test_fault();
 // test hook: 1 forces the decode kernels' y-store check to fail, 2 the
 // tensor-core kernel's (device-check build only; 0 = off)
 int test_force_check();
+// An NVTX range named for a C-ABI call, for the call's duration, when tracing
+// is on (SPEAR_NVTX=1 in the environment, or spear_set_tracing(1)); nothing otherwise
+struct TraceRange {
+  bool on;
+  explicit TraceRange(const char* name);
+  ~TraceRange();
+  TraceRange(const TraceRange&) = delete;
+  TraceRange& operator=(const TraceRange&) = delete;
+};
 // K-part flags in the workspace: 4 per (tile, part, 128-row half), tiles x parts <= SMs
 constexpr int kKFlagCapacity = 4 * 1024;
 

@@ -55,6 +55,7 @@ using namespace spear;
 
 extern "C" int spear_linear_forward_decode_noalloc(const spear_layer* layer, const uint16_t* x, int M, uint16_t* y,
                                                    float* gate_out, int* mask_count, void* stream) {
+  TraceRange trace_("spear_linear_forward_decode_noalloc");
   LayerView L;
   int rc = validate_layer(layer, &L);
   if (rc) return rc;
@@ -104,6 +105,7 @@ extern "C" int spear_linear_forward_decode_noalloc(const spear_layer* layer, con
 }
 
 extern "C" int spear_read_status_noalloc(int* device_status, void* stream) {
+  TraceRange trace_("spear_read_status_noalloc");
   if (!device_status) return set_error(SPEAR_ERR_INVALID_ARG, "device_status is NULL");
   uint8_t* scratch = nullptr;
   int rc = noalloc_scratch_ptr(&scratch);

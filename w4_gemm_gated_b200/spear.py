@@ -89,6 +89,8 @@ EXPORTS = {
     "spear_read_status_noalloc": (_i, ctypes.POINTER(_i), _vp),
     "spear_test_inject_timeout": (_i, _i, ctypes.c_longlong),
     "spear_device_checks_enabled": (_i,),
+    "spear_set_tracing": (_i, _i),
+    "spear_tracing_enabled": (_i,),
     "spear_test_force_device_check": (_i, _i),
     "spear_dispatch_choice": (_i, ctypes.POINTER(LayerStruct), _i),
     "spear_dispatch_tune": (_i, ctypes.POINTER(LayerStruct), ctypes.POINTER(_i), _i, _vp, _vp, _vp, _sz, _vp, _sz,
